@@ -1,0 +1,429 @@
+"""Benchmark: HSTU paged cache-hit attention, new tokens/s on B200.
+
+Workload (one "step"): the paged cache-hit ranking batch -- 8 users, cached histories
+U[1024, 4096] tokens, 16 new action tokens + 64 candidates per user, 4 heads x 128, page
+size 32, a 65,536-page bf16 KV pool -- through an 8-layer stack, each layer with its own
+pages: per layer hstu_kv_append (16 tokens/user) then hstu_attn_paged_fwd (80 tokens/user).
+Inputs are seeded synthetic tensors shaped like the serving benchmark of the NVIDIA HSTU
+deployment blog (KuaiRand-1K itself is not available here).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own replica of the batch
+on its own GPU (weak scaling, no collective on the data path); the time is the max over
+ranks.  The step is captured in one CUDA graph and timed with CUDA events; the 8 layers
+read ~370 MB of distinct pages per step, more than the 126 MB L2, so no flush is needed.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hstu_attention_b200 import inputs as gen  # noqa: E402
+
+METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+
+def workload_stats(layers):
+    """Algorithmic bytes and FLOPs of the paged calls, and the new-token count."""
+    tokens = int(layers[0].Tn)
+    per_layer_bytes, per_layer_flops = [], []
+    for c in layers:
+        HD = c.H * c.D
+        cached = int(np.sum(c.cached_lens))
+        # cached K and V read once; q, k, v, u of new tokens read; out written (all bf16);
+        # the page-table entries of the cached pages (int32)
+        pages = int(np.sum((c.cached_lens + c.P - 1) // c.P))
+        nbytes = cached * HD * 2 * 2 + c.Tn * HD * 2 * 5 + pages * 4
+        pairs = 0
+        for C, N, T in zip(c.cached_lens, c.new_lens, c.num_targets):
+            C, N, T = int(C), int(N), int(T)
+            hist = C + N - T
+            for r in range(N):
+                i = C + r
+                pairs += (i + 1) if i < hist else (hist + 1)
+        per_layer_bytes.append(nbytes)
+        per_layer_flops.append(4 * c.D * pairs * c.H)
+    return tokens, per_layer_bytes, per_layer_flops
+
+
+def setup_device(layers, device):
+    import torch
+
+    import hstu_attention_b200 as hb
+
+    c0 = layers[0]
+    num_pages = c0.num_pages
+    shape = (num_pages, c0.H, c0.P, c0.D)
+    kp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    vp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+
+    def d(x):
+        x = np.ascontiguousarray(x)
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+        if x.dtype == np.int64:
+            x = x.astype(np.int32)
+        return torch.from_numpy(x).to(device)
+
+    L = []
+    max_pages = max(c.max_pages for c in layers)
+    for c in layers:
+        ids = torch.from_numpy(c.page_ids.astype(np.int64)).to(device)
+        kp[ids] = d(c.pool_k)
+        vp[ids] = d(c.pool_v)
+        pt = np.full((c.B, max_pages), -1, dtype=np.int32)
+        pt[:, :c.max_pages] = c.page_table
+        L.append(dict(q=d(c.q_new), k=d(c.k_new), v=d(c.v_new), u=d(c.u_new), pt=d(pt), cl=d(c.cached_lens),
+                      nl=d(c.new_lens), nt=d(c.num_targets), rab=d(c.rab), out=torch.empty_like(d(c.q_new))))
+    p = hb.params(c0.H, c0.D, torch.bfloat16, c0.NB, c0.n_max, page_size=c0.P, num_pages=num_pages,
+                  max_pages_per_user=max_pages)
+    ws = hb.Workspace(p, c0.B, c0.Tn, c0.max_new, device=device)
+    return p, ws, kp, vp, L
+
+
+def run_step(hb, p, ws, kp, vp, L, max_new, events=None):
+    for li, t in enumerate(L):
+        hb.kv_append(p, kp, vp, t["pt"], t["k"], t["v"], t["cl"], t["nl"], t["nt"], max_new=max_new, workspace=ws)
+        if events is not None:
+            events[li][0].record()
+        hb.paged_fwd(p, t["q"], t["k"], t["v"], t["u"], kp, vp, t["pt"], t["cl"], t["nl"], t["nt"], t["rab"],
+                     max_new=max_new, workspace=ws, out=t["out"])
+        if events is not None:
+            events[li][1].record()
+
+
+def bench_prefill(hb, device, steps, warmup, peaks):
+    """Secondary line: jagged prefill (8 users, lengths U[256, 4096]) against the tensor peak."""
+    import torch
+
+    c = gen.config2_prefill()
+    d = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(device).view(torch.bfloat16)  # noqa
+    q, k, v, u = d(c.q), d(c.k), d(c.v), d(c.u)
+    off = torch.from_numpy(c.seq_offsets.astype(np.int32)).to(device)
+    nt = torch.from_numpy(c.num_targets.astype(np.int32)).to(device)
+    rab = torch.from_numpy(c.rab).to(device)
+    p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max)
+    ws = hb.Workspace(p, c.B, c.T, 4096, device=device)
+    out = torch.empty_like(q)
+    # rotate inputs larger than L2: two copies of q/k/v/u (2 x 71 MB) alternate
+    q2, k2, v2, u2 = q.clone(), k.clone(), v.clone(), u.clone()
+    sets = [(q, k, v, u), (q2, k2, v2, u2)]
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        a = sets[i % 2]
+        hb.jagged_fwd(p, *a, off, nt, rab, max_seqlen=4096, workspace=ws, out=out)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for a in sets:
+            hb.jagged_fwd(p, *a, off, nt, rab, max_seqlen=4096, workspace=ws, out=out)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (2 * steps)
+    pairs = 0
+    for L, T in zip(c.lengths, c.num_targets):
+        hist = int(L - T)
+        pairs += hist * (hist + 1) // 2 + int(T) * (hist + 1)
+    flops = 4 * c.D * pairs * c.H
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    assert ws.status() == 0
+    return {"workload": "jagged prefill: 8 users, lengths U[256,4096] (seed 1002), 64 candidates, H=4, D=128",
+            "tokens": int(c.T), "ms_per_call": ms, "tokens_per_s": c.T / (ms * 1e-3), "tflops": tf,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "traffic": None},
+            "launches_per_call": 2}
+
+
+def cpu_oracle_layer(layer, nthreads=None):
+    """Oracle time for one layer (append + paged attention of all new tokens)."""
+    import oracle
+
+    ck, cv, cpt = layer.compact_pool()
+    ck, cv = ck.copy(), cv.copy()
+    t0 = time.perf_counter()
+    oracle.kv_append(ck, cv, cpt, layer.k_new, layer.v_new, layer.cached_lens, layer.new_offsets,
+                     layer.new_lens - layer.num_targets)
+    oracle.hstu_paged(layer.q_new, layer.k_new, layer.v_new, layer.u_new, ck, cv, cpt, layer.cached_lens,
+                      layer.new_lens, layer.num_targets, layer.rab, layer.n_max, layer.eps, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks, peaks_kind = load_peaks()
+    layers_cfg = gen.CONFIG3
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+
+        layer = gen.config3_paged_layers(layers=1)[0]
+        nthreads = oracle.default_threads()
+        for _ in range(args.warmup):
+            cpu_oracle_layer(layer, nthreads)
+        times = [cpu_oracle_layer(layer, nthreads) for _ in range(args.steps)]
+        t_layer = statistics.mean(times)
+        value = layer.Tn / (t_layer * args.layers)
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "new tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_layer * args.layers * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "paged cache hit x 8 layers (one layer timed per step, scaled by 8)",
+                       "global_batch": layer.B, "seq_len": int(layer.cached_lens.max()), "parallelism": "none"},
+            "cpu_baseline": {"value": value, "unit": "new tokens/s", "cores": nthreads, "kind": "oracle",
+                             "sample": "layer 0 of the 8-layer stack: append + paged attention of all 640 new "
+                                       "tokens; new tokens/s of the stack = 640 / (8 x layer time)"},
+            "e2e": {"value": value, "unit": "new tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    import torch
+
+    import hstu_attention_b200 as hb
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    hb.load()
+
+    layers = gen.config3_paged_layers(seed=1003 + rank, layers=args.layers)
+    tokens, lbytes, lflops = workload_stats(layers)
+    p, ws, kp, vp, L = setup_device(layers, device)
+    max_new = max(c.max_new for c in layers)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        run_step(hb, p, ws, kp, vp, L, max_new)
+    torch.cuda.synchronize()
+    assert ws.status() == 0, "device status flags set during warm-up"
+
+    # capture one step (8 x append + paged attention) in a graph, with timing events around
+    # each paged attention call (external events: recorded as graph nodes)
+    events = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+              for _ in L]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run_step(hb, p, ws, kp, vp, L, max_new, events=events)
+    graph.replay()
+    torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    call_ms = []
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    elapsed_ms = e0.elapsed_time(e1)
+    # per-call durations of the last replay's paged attention calls
+    for a, b in events:
+        call_ms.append(a.elapsed_time(b))
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        dist.barrier()
+    ms_step = elapsed_ms / args.steps
+    value = tokens * world / (ms_step * 1e-3)
+    assert ws.status() == 0, "device status flags set during the timed region"
+
+    # e2e through the public API with host buffers: per step, H2D of every layer's new-token
+    # q/k/v/u and metadata from pinned memory, the step, and D2H of every layer's output.
+    host_in = []
+    for t in L:
+        host_in.append({k: t[k].cpu().pin_memory() for k in ("q", "k", "v", "u", "pt", "cl", "nl", "nt")})
+    host_out = [t["out"].cpu().pin_memory() for t in L]
+    h2d = sum(x.numel() * x.element_size() for d in host_in for x in d.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+    e_steps = max(3, args.steps // 5)
+
+    def e2e_step():
+        for t, hsrc in zip(L, host_in):
+            for k, src in hsrc.items():
+                t[k].copy_(src, non_blocking=True)
+        graph.replay()
+        for t, hdst in zip(L, host_out):
+            hdst.copy_(t["out"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    prefill = None
+    if rank == 0 and not args.no_prefill:
+        prefill = bench_prefill(hb, device, max(5, args.steps // 2), 3, peaks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        nthreads = oracle.default_threads()
+        t_layer = cpu_oracle_layer(layers[0], nthreads)
+        cpu = {"value": tokens / (t_layer * len(layers)), "unit": "new tokens/s", "cores": nthreads, "kind": "oracle",
+               "sample": "layer 0 of the 8-layer stack (append + paged attention of all 640 new tokens), "
+                         f"{t_layer:.2f} s; scaled as 640 / (8 x layer time)"}
+
+    if world > 1:
+        graph.reset() if hasattr(graph, "reset") else None
+        del graph
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    mean_call_ms = float(np.mean(call_ms))
+    mean_bytes = float(np.mean(lbytes))
+    achieved = mean_bytes / (mean_call_ms * 1e-3) / 1e9
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "new tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, shaped like the KuaiRand-1K serving config)",
+        "config": {"workload": "paged cache hit x 8 layers: 8 users, cached U[1024,4096], 16 appended + 64 "
+                               "candidates each, H=4, D=128, P=32, 65,536-page pool; per layer kv_append + "
+                               "paged attention",
+                   "global_batch": layers_cfg["B"] * world, "seq_len": int(max(int(c.cached_lens.max()) for c in layers)),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (8 layers of distinct pages, ~370 MB per step)",
+                   "graph": "one CUDA graph per step"},
+        "roofline": {"bound": "hbm", "kernel": "hstu_attn_paged_fwd (attention kernel + LayerNorm-gate kernel)",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "peak_kind": peaks_kind, "algorithmic_bytes_per_call": mean_bytes,
+                     "ms_per_call": mean_call_ms,
+                     "tflops": float(np.mean(lflops)) / (mean_call_ms * 1e-3) / 1e12},
+        "cpu_baseline": cpu,
+        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "new tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 3 * len(L),
+        "clocks": clocks,
+        "prefill": prefill,
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+"""Python binding of the HSTU B200 attention library (libhstu_b200.so, C ABI in include/hstu.h).
+
+This module only marshals arguments: it turns torch tensors into device pointers and host
+sizes and calls the C entry points of the same names.  Every step of the computation runs
+in the library's CUDA kernels.  There is no CPU fallback: if the shared library is missing
+or no GPU is present, the calls raise.
+
+    import hstu_attention_b200 as hb
+    p = hb.params(num_heads=4, head_dim=128, dtype=torch.bfloat16, num_buckets=128, n_max=4096)
+    ws = hb.Workspace(p, max_batch=8, max_tokens=20000, max_new=4096)
+    out = hb.jagged_fwd(p, q, k, v, u, seq_offsets, num_targets, rab, max_seqlen=4096, workspace=ws)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhstu_b200.so")
+_lib = None
+_lock = threading.Lock()
+
+HSTU_DTYPE_BF16 = 0
+HSTU_DTYPE_FP32 = 1
+
+DEV_BAD_PAGE = 1 << 0
+DEV_BAD_LENGTH = 1 << 1
+DEV_BAD_NMAX = 1 << 2
+DEV_TIMEOUT = 1 << 3
+DEV_SMEM_ALIGN = 1 << 4
+
+EXPORTED = (
+    "hstu_version",
+    "hstu_error_string",
+    "hstu_workspace_size",
+    "hstu_workspace_init",
+    "hstu_read_status",
+    "hstu_attn_jagged_fwd",
+    "hstu_attn_paged_fwd",
+    "hstu_kv_append",
+    "hstu_bucket_table",
+)
+
+
+class HstuParams(ctypes.Structure):
+    """Mirror of ``hstu_attn_params`` in include/hstu.h."""
+
+    _fields_ = [
+        ("num_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("num_buckets", ctypes.c_int32),
+        ("n_max", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_pages_per_user", ctypes.c_int32),
+        ("ln_eps", ctypes.c_float),
+    ]
+
+
+class HstuError(RuntimeError):
+    pass
+
+
+def load(path: Optional[str] = None):
+    """Load the shared library (raises HstuError if it is missing)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            p = path or LIB_PATH
+            if not os.path.exists(p):
+                raise HstuError(f"{p} not found: build it with `python -m hstu_attention_b200.build`")
+            lib = ctypes.CDLL(p)
+            i32, i64, sz, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+            pp = ctypes.POINTER(HstuParams)
+            lib.hstu_version.restype = ctypes.c_char_p
+            lib.hstu_version.argtypes = []
+            lib.hstu_error_string.restype = ctypes.c_char_p
+            lib.hstu_error_string.argtypes = [ctypes.c_int]
+            lib.hstu_workspace_size.restype = sz
+            lib.hstu_workspace_size.argtypes = [pp, i32, i64, i32]
+            lib.hstu_workspace_init.restype = ctypes.c_int
+            lib.hstu_workspace_init.argtypes = [vp, sz, vp]
+            lib.hstu_read_status.restype = ctypes.c_int
+            lib.hstu_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+            lib.hstu_attn_jagged_fwd.restype = ctypes.c_int
+            lib.hstu_attn_jagged_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, sz, vp]
+            lib.hstu_attn_paged_fwd.restype = ctypes.c_int
+            lib.hstu_attn_paged_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
+                                                vp, sz, vp]
+            lib.hstu_kv_append.restype = ctypes.c_int
+            lib.hstu_kv_append.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, sz, vp]
+            lib.hstu_bucket_table.restype = ctypes.c_int
+            lib.hstu_bucket_table.argtypes = [pp, i32, vp, vp]
+            _lib = lib
+    return _lib
+
+
+def version() -> str:
+    return load().hstu_version().decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = load().hstu_error_string(rc).decode()
+        raise HstuError(f"{what} failed: {msg} ({rc})")
+
+
+def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, page_size: int = 0,
+           num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5) -> HstuParams:
+    import torch
+
+    if dtype in (torch.bfloat16, "bf16"):
+        dt = HSTU_DTYPE_BF16
+    elif dtype in (torch.float32, "fp32"):
+        dt = HSTU_DTYPE_FP32
+    else:
+        raise HstuError(f"unsupported dtype {dtype}")
+    return HstuParams(num_heads, head_dim, dt, num_buckets, n_max, page_size, num_pages, max_pages_per_user,
+                      ln_eps)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise HstuError("tensor arguments must be CUDA tensors")
+    if not t.is_contiguous():
+        raise HstuError("tensor arguments must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def workspace_size(p: HstuParams, max_batch: int, max_tokens: int, max_new: int) -> int:
+    n = load().hstu_workspace_size(ctypes.byref(p), int(max_batch), int(max_tokens), int(max_new))
+    if n == 0:
+        raise HstuError("hstu_workspace_size: invalid parameters")
+    return int(n)
+
+
+class Workspace:
+    """Device scratch for the calls (status word + fp32 partial outputs), zeroed once."""
+
+    def __init__(self, p: HstuParams, max_batch: int, max_tokens: int, max_new: int, device=None, stream=None):
+        import torch
+
+        self.nbytes = workspace_size(p, max_batch, max_tokens, max_new)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        base = self.buf.data_ptr()
+        self.offset = (-base) % 256
+        self.ptr = base + self.offset
+        _check(load().hstu_workspace_init(self.ptr, self.nbytes, _stream(stream)), "hstu_workspace_init")
+
+    def status(self, clear: bool = True, stream=None) -> int:
+        flags = ctypes.c_uint32(0)
+        _check(load().hstu_read_status(self.ptr, _stream(stream), ctypes.byref(flags), int(clear)), "hstu_read_status")
+        return int(flags.value)
+
+
+def jagged_fwd(p: HstuParams, q, k, v, u, seq_offsets, num_targets, rab, *, max_seqlen: int, workspace: Workspace,
+               out=None, stream=None):
+    """hstu_attn_jagged_fwd: q/k/v/u [T, H, D]; seq_offsets [B+1] int32; num_targets [B] int32 or None;
+    rab [H, NB] fp32.  Returns out [T, H, D]."""
+    import torch
+
+    if out is None:
+        out = torch.empty_like(q)
+    B = seq_offsets.shape[0] - 1
+    rc = load().hstu_attn_jagged_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(seq_offsets),
+                                     _ptr(num_targets), _ptr(rab), _ptr(out), B, q.shape[0], int(max_seqlen),
+                                     workspace.ptr, workspace.nbytes, _stream(stream))
+    _check(rc, "hstu_attn_jagged_fwd")
+    return out
+
+
+def paged_fwd(p: HstuParams, q_new, k_new, v_new, u_new, k_pages, v_pages, page_table, cached_lens, new_lens,
+              num_targets, rab, *, max_new: int, workspace: Workspace, out=None, stream=None):
+    """hstu_attn_paged_fwd: new-token tensors [Tn, H, D]; pages [num_pages, H, P, D];
+    page_table [B, max_pages] int32; cached_lens/new_lens/num_targets [B] int32."""
+    import torch
+
+    if out is None:
+        out = torch.empty_like(q_new)
+    B = cached_lens.shape[0]
+    rc = load().hstu_attn_paged_fwd(ctypes.byref(p), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(u_new),
+                                    _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(cached_lens),
+                                    _ptr(new_lens), _ptr(num_targets), _ptr(rab), _ptr(out), B, q_new.shape[0],
+                                    int(max_new), workspace.ptr, workspace.nbytes, _stream(stream))
+    _check(rc, "hstu_attn_paged_fwd")
+    return out
+
+
+def kv_append(p: HstuParams, k_pages, v_pages, page_table, k_new, v_new, cached_lens, new_lens, num_targets, *,
+              max_new: int, workspace: Workspace, stream=None):
+    """hstu_kv_append: copy the first new_lens[b] - num_targets[b] new rows of each user into its pages."""
+    B = cached_lens.shape[0]
+    rc = load().hstu_kv_append(ctypes.byref(p), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(k_new),
+                               _ptr(v_new), _ptr(cached_lens), _ptr(new_lens), _ptr(num_targets), B,
+                               k_new.shape[0], int(max_new), workspace.ptr, workspace.nbytes, _stream(stream))
+    _check(rc, "hstu_kv_append")
+
+
+def bucket_table(p: HstuParams, n: int, stream=None):
+    """hstu_bucket_table: the library's bucket(d) for d in [0, n) as a device int32 tensor."""
+    import torch
+
+    out = torch.empty(int(n), dtype=torch.int32, device="cuda")
+    _check(load().hstu_bucket_table(ctypes.byref(p), int(n), _ptr(out), _stream(stream)), "hstu_bucket_table")
+    return out

@@ -1,0 +1,403 @@
+// api.cu -- the extern "C" entry points declared in include/hstu.h: argument validation,
+// workspace accounting, TMA descriptor encoding and kernel dispatch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <mutex>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hstu {
+
+__global__ void bucket_table_kernel(int32_t n, double ln_nmax, int32_t nb, int32_t* out)
+{
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n)
+        out[i] = bucket_of(i, ln_nmax, nb);
+}
+
+// ------------------------------------------------------------------ helpers
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_params(const hstu_attn_params* p, bool paged)
+{
+    if (!p)
+        return HSTU_ERR_INVALID_ARG;
+    if (p->num_heads < 1 || p->num_buckets < 1 || p->num_buckets > 4096 || p->n_max < 1)
+        return HSTU_ERR_INVALID_ARG;
+    if (!(p->ln_eps >= 0.0f) || !isfinite(p->ln_eps))
+        return HSTU_ERR_INVALID_ARG;
+    if (p->dtype != HSTU_DTYPE_BF16 && p->dtype != HSTU_DTYPE_FP32)
+        return HSTU_ERR_UNSUPPORTED;
+    if (p->head_dim != 32 && p->head_dim != 64 && p->head_dim != 128)
+        return HSTU_ERR_UNSUPPORTED;
+    if ((int64_t)p->num_heads * p->head_dim > 2048)
+        return HSTU_ERR_UNSUPPORTED;
+    if (paged) {
+        const int P = p->page_size;
+        if (P != 8 && P != 16 && P != 32 && P != 64 && P != 128)
+            return HSTU_ERR_UNSUPPORTED;
+        if (p->num_pages < 1 || p->max_pages_per_user < 1)
+            return HSTU_ERR_INVALID_ARG;
+        if ((int64_t)p->num_pages * p->num_heads * P >= (int64_t)1 << 31)
+            return HSTU_ERR_UNSUPPORTED;     // TMA row coordinates are 32-bit
+        if ((int64_t)p->max_pages_per_user * P >= (int64_t)1 << 30)
+            return HSTU_ERR_UNSUPPORTED;
+    }
+    return HSTU_OK;
+}
+
+static int esize_of(const hstu_attn_params* p) { return p->dtype == HSTU_DTYPE_FP32 ? 4 : 2; }
+
+static bool use_tc(const hstu_attn_params* p) { return p->dtype == HSTU_DTYPE_BF16 && p->head_dim == 128; }
+
+static int num_sms()
+{
+    static int cached = 0;
+    if (cached == 0) {
+        int dev = 0, n = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+            cached = n;
+        else
+            return 148;
+    }
+    return cached;
+}
+
+// Split of each (user, head, query block)'s keys over CTAs for the paged tensor-core path:
+// enough CTAs to cover the SMs once, at most kMaxSplits.
+static int paged_splits(const hstu_attn_params* p, int32_t B, int32_t max_new)
+{
+    const int64_t qblocks = (max_new + 127) / 128;
+    const int64_t units = (int64_t)B * p->num_heads * (qblocks > 0 ? qblocks : 1);
+    int64_t s = units > 0 ? num_sms() / units : 1;
+    if (s < 1)
+        s = 1;
+    if (s > kMaxSplits)
+        s = kMaxSplits;
+    return (int)s;
+}
+
+static size_t partial_bytes(const hstu_attn_params* p, int splits, int64_t tokens)
+{
+    return (size_t)splits * (size_t)tokens * (size_t)p->num_heads * (size_t)p->head_dim * sizeof(float);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// [rows][H][D] bf16 token rows; box = 64 channels x 1 head x 128 rows, 128B swizzle.
+static bool encode_rows(CUtensorMap* m, const void* base, int64_t rows, int32_t H, int32_t D)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    cuuint32_t box[3] = {64, 1, 128};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [num_pages*H*P][D] bf16 page rows; box = 64 channels x P rows, 128B swizzle.
+static bool encode_pages(CUtensorMap* m, const void* base, int64_t rows, int32_t D, int32_t P)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)P};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int finish(cudaStream_t)
+{
+    return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+static constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s per in-kernel wait
+
+}  // namespace hstu
+
+using namespace hstu;
+
+extern "C" {
+
+const char* hstu_version(void) { return "hstu_b200 0.1 (sm_100a)"; }
+
+const char* hstu_error_string(int code)
+{
+    switch (code) {
+    case HSTU_OK: return "ok";
+    case HSTU_ERR_INVALID_ARG: return "invalid argument";
+    case HSTU_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case HSTU_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case HSTU_ERR_CUDA: return "CUDA error";
+    default: return "unknown error";
+    }
+}
+
+size_t hstu_workspace_size(const hstu_attn_params* params, int32_t max_batch, int64_t max_tokens, int32_t max_new)
+{
+    if (check_params(params, false) != HSTU_OK || max_batch < 0 || max_tokens < 0 || max_new < 0)
+        return 0;
+    int splits = 1;
+    if (use_tc(params))
+        splits = paged_splits(params, max_batch > 0 ? max_batch : 1, max_new);
+    size_t bytes = kStatusBytes + partial_bytes(params, splits, max_tokens);
+    return (bytes + 255) & ~(size_t)255;
+}
+
+int hstu_workspace_init(void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!workspace || workspace_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (cudaMemsetAsync(workspace, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    return HSTU_OK;
+}
+
+int hstu_read_status(void* workspace, void* stream, uint32_t* flags_out, int clear)
+{
+    if (!workspace || !flags_out)
+        return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, workspace, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    *flags_out = v;
+    if (clear && cudaMemset(workspace, 0, sizeof v) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    return HSTU_OK;
+}
+
+int hstu_bucket_table(const hstu_attn_params* params, int32_t n, int32_t* table_out, void* stream)
+{
+    if (check_params(params, false) != HSTU_OK || n < 0 || (n > 0 && !table_out))
+        return HSTU_ERR_INVALID_ARG;
+    if (n == 0)
+        return HSTU_OK;
+    const double ln_nmax = log((double)params->n_max);
+    bucket_table_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(n, ln_nmax,
+                                                                                        params->num_buckets, table_out);
+    return finish(static_cast<cudaStream_t>(stream));
+}
+
+int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages, const int32_t* page_table,
+                   const void* k_new, const void* v_new, const int32_t* cached_lens, const int32_t* new_lens,
+                   const int32_t* num_targets, int32_t B, int64_t total_new, int32_t max_new, void* workspace,
+                   size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, true);
+    if (rc != HSTU_OK)
+        return rc;
+    if (B < 0 || max_new < 0 || total_new < 0)
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (B == 0 || max_new == 0 || total_new == 0)
+        return HSTU_OK;
+    if (!k_pages || !v_pages || !page_table || !k_new || !v_new || !cached_lens || !new_lens)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(k_pages) || !aligned16(v_pages) || !aligned16(k_new) || !aligned16(v_new))
+        return HSTU_ERR_INVALID_ARG;
+    launch_kv_append(k_pages, v_pages, page_table, k_new, v_new, cached_lens, new_lens, num_targets, B, total_new,
+                     params->num_heads, params->head_dim, esize_of(params), params->page_size, params->num_pages,
+                     params->max_pages_per_user, max_new, workspace, static_cast<cudaStream_t>(stream));
+    return finish(static_cast<cudaStream_t>(stream));
+}
+
+int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const void* k, const void* v, const void* u,
+                         const int32_t* seq_offsets, const int32_t* num_targets, const float* rab, void* out,
+                         int32_t B, int64_t total_tokens, int32_t max_seqlen, void* workspace,
+                         size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, false);
+    if (rc != HSTU_OK)
+        return rc;
+    if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (B == 0 || total_tokens == 0 || max_seqlen == 0)
+        return HSTU_OK;
+    if (!q || !k || !v || !u || !out || !seq_offsets || !rab)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out))
+        return HSTU_ERR_INVALID_ARG;
+    if (workspace_bytes < kStatusBytes + partial_bytes(params, 1, total_tokens))
+        return HSTU_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const double ln_nmax = log((double)params->n_max);
+    const bool fp32 = params->dtype == HSTU_DTYPE_FP32;
+    if (use_tc(params)) {
+        TcMaps m;
+        if (!encode_rows(&m.q, q, total_tokens, params->num_heads, 128) ||
+            !encode_rows(&m.k, k, total_tokens, params->num_heads, 128) ||
+            !encode_rows(&m.v, v, total_tokens, params->num_heads, 128))
+            return HSTU_ERR_CUDA;
+        m.kp = m.k;
+        m.vp = m.v;
+        TcArgs a{};
+        a.seq_offsets = seq_offsets;
+        a.num_targets = num_targets;
+        a.rab = rab;
+        a.ws = workspace;
+        a.total_tokens = total_tokens;
+        a.max_len = max_seqlen;
+        a.H = params->num_heads;
+        a.NB = params->num_buckets;
+        a.n_max = params->n_max;
+        a.P = 1;
+        a.num_pages = 0;
+        a.max_pages = 0;
+        a.splits = 1;
+        a.qblocks = (max_seqlen + 127) / 128;
+        a.ln_nmax = ln_nmax;
+        a.inv_n = (float)(1.0 / (double)params->n_max);
+        a.timeout_ns = kTimeoutNs;
+        launch_attn_tc(m, a, false, B, s);
+    } else {
+        SimtArgs a{};
+        a.q = q;
+        a.k = k;
+        a.v = v;
+        a.seq_offsets = seq_offsets;
+        a.num_targets = num_targets;
+        a.rab = rab;
+        a.ws = workspace;
+        a.total_tokens = total_tokens;
+        a.max_len = max_seqlen;
+        a.H = params->num_heads;
+        a.D = params->head_dim;
+        a.NB = params->num_buckets;
+        a.n_max = params->n_max;
+        a.P = 1;
+        a.ln_nmax = ln_nmax;
+        launch_attn_simt(a, false, fp32, B, s);
+    }
+    launch_ln_gate(partials(workspace), 1, total_tokens, params->num_heads * params->head_dim, u, out, fp32,
+                   params->ln_eps, s);
+    return finish(s);
+}
+
+int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const void* k_new, const void* v_new,
+                        const void* u_new, const void* k_pages, const void* v_pages, const int32_t* page_table,
+                        const int32_t* cached_lens, const int32_t* new_lens, const int32_t* num_targets,
+                        const float* rab, void* out, int32_t B, int64_t total_new, int32_t max_new, void* workspace,
+                        size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, true);
+    if (rc != HSTU_OK)
+        return rc;
+    if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (B == 0 || total_new == 0 || max_new == 0)
+        return HSTU_OK;
+    if (!q_new || !k_new || !v_new || !u_new || !k_pages || !v_pages || !page_table || !cached_lens || !new_lens ||
+        !rab || !out)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(u_new) || !aligned16(k_pages) ||
+        !aligned16(v_pages) || !aligned16(out))
+        return HSTU_ERR_INVALID_ARG;
+    const size_t one = partial_bytes(params, 1, total_new);
+    if (workspace_bytes < kStatusBytes + one)
+        return HSTU_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const double ln_nmax = log((double)params->n_max);
+    const bool fp32 = params->dtype == HSTU_DTYPE_FP32;
+    int splits = 1;
+    if (use_tc(params)) {
+        splits = paged_splits(params, B, max_new);
+        const int fit = (int)((workspace_bytes - kStatusBytes) / one);
+        if (splits > fit)
+            splits = fit;
+        TcMaps m;
+        const int64_t page_rows = (int64_t)params->num_pages * params->num_heads * params->page_size;
+        if (!encode_rows(&m.q, q_new, total_new, params->num_heads, 128) ||
+            !encode_rows(&m.k, k_new, total_new, params->num_heads, 128) ||
+            !encode_rows(&m.v, v_new, total_new, params->num_heads, 128) ||
+            !encode_pages(&m.kp, k_pages, page_rows, 128, params->page_size) ||
+            !encode_pages(&m.vp, v_pages, page_rows, 128, params->page_size))
+            return HSTU_ERR_CUDA;
+        TcArgs a{};
+        a.cached_lens = cached_lens;
+        a.new_lens = new_lens;
+        a.num_targets = num_targets;
+        a.page_table = page_table;
+        a.rab = rab;
+        a.ws = workspace;
+        a.total_tokens = total_new;
+        a.max_len = max_new;
+        a.H = params->num_heads;
+        a.NB = params->num_buckets;
+        a.n_max = params->n_max;
+        a.P = params->page_size;
+        a.num_pages = params->num_pages;
+        a.max_pages = params->max_pages_per_user;
+        a.splits = splits;
+        a.qblocks = (max_new + 127) / 128;
+        a.ln_nmax = ln_nmax;
+        a.inv_n = (float)(1.0 / (double)params->n_max);
+        a.timeout_ns = kTimeoutNs;
+        launch_attn_tc(m, a, true, B, s);
+    } else {
+        SimtArgs a{};
+        a.q = q_new;
+        a.k = k_new;
+        a.v = v_new;
+        a.k_pages = k_pages;
+        a.v_pages = v_pages;
+        a.page_table = page_table;
+        a.cached_lens = cached_lens;
+        a.new_lens = new_lens;
+        a.num_targets = num_targets;
+        a.rab = rab;
+        a.ws = workspace;
+        a.total_tokens = total_new;
+        a.max_len = max_new;
+        a.H = params->num_heads;
+        a.D = params->head_dim;
+        a.NB = params->num_buckets;
+        a.n_max = params->n_max;
+        a.P = params->page_size;
+        a.num_pages = params->num_pages;
+        a.max_pages = params->max_pages_per_user;
+        a.ln_nmax = ln_nmax;
+        launch_attn_simt(a, true, fp32, B, s);
+    }
+    launch_ln_gate(partials(workspace), splits, total_new, params->num_heads * params->head_dim, u_new, out, fp32,
+                   params->ln_eps, s);
+    return finish(s);
+}
+
+}  // extern "C"

@@ -1,0 +1,461 @@
+// attn_tc.cu -- HSTU attention on Blackwell tensor cores (bf16 in, fp32 accumulate, D = 128).
+//
+// What it computes (per user b, head h): for a block of 128 query rows and the key tiles the
+// block may see,
+//     S = Q K^T                               tcgen05.mma, accumulator in tensor memory
+//     P = allowed ? SiLU(S + rab[h][bucket(i-j)]) / n_max : 0      (registers, -> bf16)
+//     O += P V                                tcgen05.mma, accumulator in tensor memory
+// SiLU weighting replaces softmax, so there is no running max or row sum and key tiles can be
+// split across CTAs and summed afterwards (aitrends.kr summary, section "HSTU의 순차 모델링";
+// news.bpdata.com, section "HSTU").  Keys of the paged layout come from the per-user page
+// table for positions below cached_len and from the new-token rows after that (NVIDIA blog
+// "Deploying an HSTU Generative Recommender with NVIDIA Dynamo-Triton", section "Why serving
+// large sequential recommenders is hard": the attention kernel reads K/V from the paged
+// cache).  O (fp32) goes to the workspace; combine.cu applies LayerNorm(O) * U.
+//
+// CTA roles (384 threads):
+//   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring.  Paged tiles
+//               are gathered page by page (one TMA box of P rows per page and channel half).
+//   warp 1      allocates 512 TMEM columns; lane 0 issues all MMAs:
+//               S_t = Q K_t^T into S buffer t%2, then O += P_{t-1} V_{t-1}, so the pointwise
+//               work on S_t overlaps the P V product of the previous tile.
+//   warps 4-11  two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
+//               warp w%4 owns TMEM lanes (= query rows) [32(w%4), +32).  They load S from
+//               TMEM, add the bias, mask, apply SiLU/n_max, write bf16 P into shared memory in
+//               the 128-byte-swizzled K-major layout the MMA reads, and at the end move O
+//               from TMEM to the workspace.
+// Shared memory (1024-byte aligned, 128B swizzle everywhere):
+//   Q 32 KB | 2 x (K 32 KB + V 32 KB) | P 32 KB | 2 bias windows | mbarriers
+// Every wait is bounded (HSTU_DEV_TIMEOUT) so a logic error cannot hang the GPU.
+#include "common.cuh"
+#include "sm100.cuh"
+#include "kernels.cuh"
+
+namespace hstu {
+using namespace sm100;
+
+constexpr int kTcD = 128;
+constexpr int kTile = 128;                    // query rows per CTA and keys per tile
+constexpr int kStages = 2;
+constexpr int kTcThreads = 384;
+constexpr uint32_t kHalf = 128 * 128;         // 128 rows x 128 bytes = 16 KB (one swizzle column)
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffStage = 2 * kHalf;     // stage s at kOffStage + s * kStageBytes
+constexpr uint32_t kStageBytes = 4 * kHalf;   // K halves then V halves
+constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffWin = kOffP + 2 * kHalf;
+constexpr uint32_t kWinFloats = 256;
+constexpr uint32_t kOffBar = kOffWin + 2 * kWinFloats * 4;
+constexpr int kNumBars = 14;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemUsed = kOffMisc + 16;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;     // slack to align the base to 1024
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct TileGeo {
+    int32_t j0;       // absolute position of key row 0 of the tile
+    int32_t kvend;    // keys at positions >= kvend are not valid data for this tile
+    bool cached;      // keys come from pages
+};
+
+__device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t ct, int32_t C, int32_t L)
+{
+    TileGeo g;
+    if (t < ct) {
+        g.j0 = t * kTile;
+        g.kvend = C;
+        g.cached = true;
+    } else {
+        g.j0 = C + (t - ct) * kTile;
+        g.kvend = L;
+        g.cached = false;
+    }
+    return g;
+}
+
+template <bool kPaged>
+__global__ void __launch_bounds__(kTcThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+               const __grid_constant__ CUtensorMap tm_vp, const TcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ UserGeom sG;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.z, h = blockIdx.y;
+    const int split = blockIdx.x % a.splits;
+    const int qblk = a.qblocks - 1 - (int)(blockIdx.x / a.splits);     // heaviest query blocks first
+
+    if (warp == 0) {
+        UserGeom g = kPaged ? paged_geom(a.cached_lens, a.new_lens, a.num_targets, b, a.total_tokens, a.max_len,
+                                         a.max_pages * a.P, a.n_max, a.ws, blockIdx.x == 0 && h == 0)
+                            : jagged_geom(a.seq_offsets, a.num_targets, b, a.total_tokens, a.max_len, a.n_max,
+                                          a.ws, blockIdx.x == 0 && h == 0);
+        if (lane == 0)
+            sG = g;
+    }
+    __syncthreads();
+    const UserGeom g = sG;
+    const int32_t qrow0 = qblk * kTile;
+    if (qrow0 >= g.N)
+        return;                                               // no queries here (uniform)
+
+    const int32_t i0 = g.C + qrow0;                           // absolute position of row 0
+    const int32_t last_q = min(g.N, qrow0 + kTile) - 1;
+    const int32_t kend = min(g.L, g.C + last_q + 1);          // later keys are never visible
+    const int32_t ct = kPaged ? (g.C + kTile - 1) / kTile : 0;
+    const int32_t nnew = kend > g.C ? (kend - g.C + kTile - 1) / kTile : 0;
+    const int32_t ntot = ct + nnew;
+    const int32_t t_begin = (int32_t)(((int64_t)ntot * split) / a.splits);
+    const int32_t t_end = (int32_t)(((int64_t)ntot * (split + 1)) / a.splits);
+    const int32_t n = g.ok ? t_end - t_begin : 0;
+    const int64_t HD = (int64_t)a.H * kTcD;
+    float* part = partials(a.ws) + (int64_t)split * a.total_tokens * HD;
+
+    if (n <= 0) {
+        // nothing to accumulate: this split's partial rows are zero
+        for (int x = threadIdx.x; x < kTile * (kTcD / 4); x += kTcThreads) {
+            const int r = x / (kTcD / 4), c4 = x % (kTcD / 4);
+            if (qrow0 + r < g.N)
+                reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + r) * HD + (int64_t)h * kTcD)[c4] =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- shared memory carve-up
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw_u32 & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t sbase = raw_u32 + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* q_full = bars + 0;
+    uint64_t* k_full = bars + 1;      // [2]
+    uint64_t* v_full = bars + 3;      // [2]
+    uint64_t* kv_empty = bars + 5;    // [2]
+    uint64_t* s_full = bars + 7;      // [2]
+    uint64_t* s_empty = bars + 9;     // [2]
+    uint64_t* p_full = bars + 11;
+    uint64_t* p_empty = bars + 12;
+    uint64_t* o_full = bars + 13;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    float* win = reinterpret_cast<float*>(smem + kOffWin);
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], 256);
+        }
+        mbar_init(p_full, 256);
+        mbar_init(p_empty, 1);
+        mbar_init(o_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint64_t tmo = a.timeout_ns;
+
+    if (warp == 0 && lane == 0) {
+        // ============================================================ TMA producer
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        if (kPaged) {
+            tma_prefetch_desc(&tm_kp);
+            tma_prefetch_desc(&tm_vp);
+        }
+        mbar_arrive_expect_tx(q_full, 2 * kHalf);
+        for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(&tm_q, sbase + kOffQ + hf * kHalf, q_full, hf * 64, h, (int32_t)(g.tok0 + qrow0));
+        int issued = 0;
+        for (int t = 0; t < n; ++t) {
+            const int st = t % kStages;
+            const uint32_t kph = (t / kStages) & 1;
+            if (t >= kStages && !mbar_wait(&kv_empty[st], kph ^ 1, abort_flag, tmo))
+                break;
+            const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
+            const uint32_t kdst = sbase + kOffStage + st * kStageBytes;
+            const uint32_t vdst = kdst + 2 * kHalf;
+            if (kPaged && tg.cached) {
+                const int P = a.P;
+                const int lp0 = tg.j0 / P;
+                const int npg = kTile / P;
+                uint32_t bytes = 0;
+                int32_t pages[kTile / 8];
+                for (int k = 0; k < npg; ++k) {
+                    const int lp = lp0 + k;
+                    int32_t pg = -1;
+                    if (lp * P < g.C) {
+                        pg = a.page_table[(int64_t)b * a.max_pages + lp];
+                        if (pg < 0 || pg >= a.num_pages) {
+                            set_flag(a.ws, HSTU_DEV_BAD_PAGE);
+                            pg = -1;
+                        } else {
+                            bytes += (uint32_t)P * 128u * 2u;
+                        }
+                    }
+                    pages[k] = pg;
+                }
+                mbar_arrive_expect_tx(&k_full[st], bytes);
+                for (int k = 0; k < npg; ++k) {
+                    if (pages[k] < 0)
+                        continue;
+                    const int32_t row = (pages[k] * a.H + h) * P;
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_load_2d(&tm_kp, kdst + hf * kHalf + k * P * 128, &k_full[st], hf * 64, row);
+                }
+                mbar_arrive_expect_tx(&v_full[st], bytes);
+                for (int k = 0; k < npg; ++k) {
+                    if (pages[k] < 0)
+                        continue;
+                    const int32_t row = (pages[k] * a.H + h) * P;
+                    for (int hf = 0; hf < 2; ++hf)
+                        tma_load_2d(&tm_vp, vdst + hf * kHalf + k * P * 128, &v_full[st], hf * 64, row);
+                }
+            } else {
+                const int32_t row = (int32_t)(g.key_row0 + (tg.j0 - g.C));
+                mbar_arrive_expect_tx(&k_full[st], 2 * kHalf);
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(&tm_k, kdst + hf * kHalf, &k_full[st], hf * 64, h, row);
+                mbar_arrive_expect_tx(&v_full[st], 2 * kHalf);
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(&tm_v, vdst + hf * kHalf, &v_full[st], hf * 64, h, row);
+            }
+            issued = t + 1;
+        }
+        // drain: loads still in flight must land before the CTA may exit (a local flag, so
+        // the drain itself never raises the CTA-wide abort)
+        volatile int never = 0;
+        mbar_wait(q_full, 0, &never, tmo);
+        for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t) {
+            const int st = t % kStages;
+            const uint32_t kph = (t / kStages) & 1;
+            mbar_wait(&k_full[st], kph, &never, tmo);
+            mbar_wait(&v_full[st], kph, &never, tmo);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ============================================================ MMA issuer
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+        const uint32_t qbase = sbase + kOffQ;
+        const uint32_t pbase = sbase + kOffP;
+        bool ok = mbar_wait(q_full, 0, abort_flag, tmo);
+        auto issue_pv = [&](int u) -> bool {
+            const int st = u % kStages;
+            const uint32_t kph = (u / kStages) & 1;
+            if (!mbar_wait(p_full, u & 1, abort_flag, tmo))
+                return false;
+            if (!mbar_wait(&v_full[st], kph, abort_flag, tmo))
+                return false;
+            tc_fence_after();
+            const uint32_t vbase = sbase + kOffStage + st * kStageBytes + 2 * kHalf;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = smem_desc_sw128(pbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, kHalf, 1024);
+                umma_bf16_ss(tmem + kColO, ad, bd, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(p_empty);
+            umma_commit(&kv_empty[st]);
+            return true;
+        };
+        for (int t = 0; ok && t < n; ++t) {
+            const int st = t % kStages;
+            const uint32_t kph = (t / kStages) & 1;
+            const int sb = t & 1;
+            const uint32_t sph = (t >> 1) & 1;
+            if (!mbar_wait(&k_full[st], kph, abort_flag, tmo)) {
+                ok = false;
+                break;
+            }
+            if (t >= 2 && !mbar_wait(&s_empty[sb], sph ^ 1, abort_flag, tmo)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t kbase = sbase + kOffStage + st * kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t ad = smem_desc_sw128(qbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+                umma_bf16_ss(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[sb]);
+            if (t >= 1 && !issue_pv(t - 1)) {
+                ok = false;
+                break;
+            }
+        }
+        if (ok)
+            ok = issue_pv(n - 1);
+        // o_full fires once every MMA issued so far has completed (also on the abort path,
+        // so tensor memory is idle before it is released)
+        umma_commit(o_full);
+        volatile int never = 0;
+        mbar_wait(o_full, 0, &never, tmo);
+    } else if (warp >= 4) {
+        // ============================================================ pointwise + epilogue
+        const int pt = threadIdx.x - 128;                 // 0..255
+        const int wg = (warp - 4) >> 2;                   // key-column half
+        const int r = ((warp & 3) << 5) + lane;           // query row in the block (= TMEM lane)
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool row_valid = qrow0 + r < g.N;
+        const int32_t i_abs = i0 + r;
+        const int32_t lim_row = row_valid ? min(i_abs + 1, g.hist) : -1;
+        const float half_inv_n = 0.5f * a.inv_n;
+        const float* rab_h = a.rab + (int64_t)h * a.NB;
+        uint8_t* pbuf = smem + kOffP + wg * kHalf + r * 128;
+        bool ok = true;
+        for (int t = 0; t < n; ++t) {
+            const int st = t % kStages;
+            const uint32_t kph = (t / kStages) & 1;
+            const int sb = t & 1;
+            const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
+            float* w_t = win + sb * kWinFloats;
+            if (pt < 2 * kTile - 1) {
+                const int64_t dist = (int64_t)i0 - tg.j0 - (kTile - 1) + pt;
+                w_t[pt] = dist >= 0 ? rab_h[bucket_of(dist, a.ln_nmax, a.NB)] : 0.f;
+            }
+            named_barrier_sync(1, 256);
+            ok = ok && mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
+                continue;
+            tc_fence_after();
+            uint32_t sv[2][32];
+            const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0) + wg * 64;
+            tmem_ld_32x32b_x32(scol, sv[0]);
+            tmem_ld_32x32b_x32(scol + 32, sv[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&s_empty[sb]);
+
+            const bool full = (qrow0 + kTile - 1 < g.N) && (tg.j0 + kTile - 1 < tg.kvend) &&
+                              (tg.j0 + kTile - 1 <= i0) && (tg.j0 + kTile - 1 < g.hist);
+            const int32_t lim = min(lim_row, tg.kvend);
+            const int32_t diag = (row_valid && !tg.cached) ? i_abs : -1;
+            const int jc0 = tg.j0 + wg * 64;                  // key position of column 0 of this half
+            const float* wrow = w_t + r + (kTile - 1) - wg * 64;   // wrow[-c] = bias at column c
+            uint32_t packed[32];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+                // SiLU(x) / n_max = hx * (1 + tanh(x / 2)) with hx = x / (2 n_max)
+                const float x0 = __uint_as_float(sv[c >> 5][c & 31]) + wrow[-c];
+                const float x1 = __uint_as_float(sv[(c + 1) >> 5][(c + 1) & 31]) + wrow[-(c + 1)];
+                const float h0 = x0 * half_inv_n, h1 = x1 * half_inv_n;
+                float w0 = fmaf(h0, tanh_approx(0.5f * x0), h0);
+                float w1 = fmaf(h1, tanh_approx(0.5f * x1), h1);
+                if (!full) {
+                    const int j = jc0 + c;
+                    w0 = ((j < lim) || (j == diag)) ? w0 : 0.f;
+                    w1 = ((j + 1 < lim) || (j + 1 == diag)) ? w1 : 0.f;
+                }
+                __nv_bfloat162 p2 = __floats2bfloat162_rn(w0, w1);
+                packed[c >> 1] = *reinterpret_cast<uint32_t*>(&p2);
+            }
+            if (t >= 1) {
+                ok = ok && mbar_wait(p_empty, (t - 1) & 1, abort_flag, tmo);
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            if (!ok)
+                continue;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                uint4 v4 = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                *reinterpret_cast<uint4*>(pbuf + ((q ^ (r & 7)) << 4)) = v4;
+            }
+            const int vz = tg.kvend - tg.j0;                   // valid key rows in this tile
+            if (vz < kTile) {
+                ok = ok && mbar_wait(&v_full[st], kph, abort_flag, tmo);
+                if (ok) {
+                    uint8_t* vt = smem + kOffStage + st * kStageBytes + 2 * kHalf;
+                    const int first = vz > 0 ? vz : 0;
+                    const int nchunks = (kTile - first) * 16;
+                    for (int x = pt; x < nchunks; x += 256) {
+                        const int row = first + (x >> 4), hf = (x >> 3) & 1, ch = x & 7;
+                        *reinterpret_cast<uint4*>(vt + hf * kHalf + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
+            if (ok) {
+                fence_proxy_async_smem();
+                mbar_arrive(p_full);
+            }
+        }
+        // ------------------------------------------------------------ epilogue: O -> workspace
+        ok = ok && mbar_wait(o_full, 0, abort_flag, tmo);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            uint32_t ov[2][32];
+            const uint32_t ocol = tmem + lane_base + kColO + wg * 64;
+            tmem_ld_32x32b_x32(ocol, ov[0]);
+            tmem_ld_32x32b_x32(ocol + 32, ov[1]);
+            tmem_wait_ld();
+            if (row_valid) {
+                float4* dst = reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + r) * HD + (int64_t)h * kTcD + wg * 64);
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4) {
+                    const int c = c4 * 4;
+                    dst[c4] = make_float4(__uint_as_float(ov[c >> 5][c & 31]), __uint_as_float(ov[c >> 5][(c & 31) + 1]),
+                                          __uint_as_float(ov[c >> 5][(c & 31) + 2]),
+                                          __uint_as_float(ov[c >> 5][(c & 31) + 3]));
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag)
+        set_flag(a.ws, HSTU_DEV_TIMEOUT);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+void launch_attn_tc(const TcMaps& m, const TcArgs& a, bool paged, int32_t B, cudaStream_t stream)
+{
+    static bool attr_set[2] = {false, false};
+    const int grid_x = a.qblocks * a.splits;
+    if (B <= 0 || grid_x <= 0)
+        return;
+    dim3 grid(grid_x, a.H, B);
+    if (paged) {
+        if (!attr_set[1]) {
+            cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            attr_set[1] = true;
+        }
+        attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, a);
+    } else {
+        if (!attr_set[0]) {
+            cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            attr_set[0] = true;
+        }
+        attn_tc_kernel<false><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, a);
+    }
+}
+
+}  // namespace hstu

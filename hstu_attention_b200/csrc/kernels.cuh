@@ -1,0 +1,56 @@
+// kernels.cuh -- launch interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hstu {
+
+struct SimtArgs {
+    const void *q, *k, *v;                 // jagged rows, or q_new / k_new / v_new
+    const void *k_pages, *v_pages;         // paged only
+    const int32_t* page_table;
+    const int32_t* seq_offsets;            // jagged
+    const int32_t *cached_lens, *new_lens; // paged
+    const int32_t* num_targets;
+    const float* rab;
+    void* ws;
+    int64_t total_tokens;                  // jagged: all tokens; paged: all new tokens
+    int32_t max_len;                       // jagged: max_seqlen; paged: max_new
+    int32_t H, D, NB, n_max, P, num_pages, max_pages;
+    double ln_nmax;
+};
+
+struct TcArgs {
+    const int32_t* seq_offsets;
+    const int32_t* cached_lens;
+    const int32_t* new_lens;
+    const int32_t* num_targets;
+    const int32_t* page_table;
+    const float* rab;
+    void* ws;
+    int64_t total_tokens;   // rows of q/k/v/u (jagged) or of the new-token arrays (paged)
+    int32_t max_len;        // jagged: max_seqlen; paged: max_new
+    int32_t H, NB, n_max, P, num_pages, max_pages, splits, qblocks;
+    double ln_nmax;
+    float inv_n;
+    uint64_t timeout_ns;
+};
+
+struct TcMaps {
+    CUtensorMap q, k, v, kp, vp;
+};
+
+void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, const void* k_new,
+                      const void* v_new, const int32_t* cached_lens, const int32_t* new_lens,
+                      const int32_t* num_targets, int32_t B, int64_t total_new, int32_t H, int32_t D,
+                      int32_t esize,
+                      int32_t P, int32_t num_pages, int32_t max_pages, int32_t max_new, void* ws,
+                      cudaStream_t stream);
+void launch_ln_gate(const float* part, int32_t S, int64_t ntok, int32_t HD, const void* u, void* out, bool fp32,
+                    float eps, cudaStream_t stream);
+void launch_attn_simt(const SimtArgs& a, bool paged, bool fp32, int32_t B, cudaStream_t stream);
+void launch_attn_tc(const TcMaps& m, const TcArgs& a, bool paged, int32_t B, cudaStream_t stream);
+
+}  // namespace hstu

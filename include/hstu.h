@@ -1,0 +1,188 @@
+/*
+ * hstu.h -- C ABI of the B200 (sm_100a) HSTU attention library.
+ *
+ * The operation (per user b, head h, query position i, key position j of the user's sequence):
+ *
+ *   Hist_b      = L_b - num_targets[b]           history length; the last num_targets[b]
+ *                                                tokens are the ranking candidates
+ *   allowed     = (j <= i and j < Hist_b) or (j == i)
+ *                 causal over the history; a candidate sees the whole history and itself,
+ *                 never another candidate
+ *   s           = sum_c q[i,h,c] * k[j,h,c] + rab[h][bucket(i - j)]
+ *   w           = allowed ? s * sigmoid(s) / n_max : 0          (SiLU weighting, no softmax)
+ *   o[i,h,:]    = sum_j w * v[j,h,:]
+ *   out[i,h,c]  = (o[i,h,c] - mean_i) / sqrt(var_i + ln_eps) * u[i,h,c]
+ *                 mean_i, var_i (biased) over all H*D values of token i
+ *
+ *   bucket(0) = 0;  bucket(d) = min(NB-1, 1 + floor((NB-1) * ln(d) / ln(n_max))) for d >= 1
+ *
+ * Sources: HSTU swaps softmax for SiLU-based weighting, adds a relative attention bias and
+ * gates elementwise before the output projection (aitrends.kr summary of the NVIDIA
+ * recsys post, section "HSTU의 순차 모델링"; news.bpdata.com, section "HSTU").  Inputs are
+ * jagged per-user sequences; in serving the HSTU attention kernel reads the user's history
+ * K/V from a paged GPU KV table and only the new tokens are computed and appended (NVIDIA
+ * blog "Deploying an HSTU Generative Recommender with NVIDIA Dynamo-Triton", sections
+ * "Why serving large sequential recommenders is hard" and "Benefits").  The pages leave the
+ * bias bucketing, the 1/n_max scale, the LayerNorm axis and eps open; the readings above
+ * are this library's definition.
+ *
+ * Conventions for every call
+ *   - All tensor arguments are DEVICE pointers, caller-owned, 16-byte aligned, row-major.
+ *     Token tensors are [tokens][H][D] (D contiguous).  Pages are [num_pages][H][P][D].
+ *   - Element type: params->dtype (HSTU_DTYPE_BF16 or HSTU_DTYPE_FP32) for q, k, v, u,
+ *     pages and out.  rab is always fp32 [H][NB].  Index arrays are int32.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream).  They do not synchronise and allocate no device memory.
+ *   - Scratch lives in a caller-provided workspace of at least hstu_workspace_size()
+ *     bytes, 256-byte aligned, zeroed once with hstu_workspace_init() before first use.
+ *     One workspace must not be used by two calls that may run concurrently.
+ *   - Host-detectable argument errors return a negative hstu_status_code and launch
+ *     nothing.  Errors only the device can see (a page id out of range, lengths that do
+ *     not fit, offsets that decrease, a kernel wait that timed out) set bits of a status
+ *     word inside the workspace; the offending user's output rows are written as zeros
+ *     and no kernel traps.  Read (and clear) that word with hstu_read_status().
+ */
+#ifndef HSTU_B200_H
+#define HSTU_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HSTU_OK = 0,
+    HSTU_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misaligned pointer */
+    HSTU_ERR_UNSUPPORTED = -2,  /* a shape this build does not implement */
+    HSTU_ERR_WORKSPACE = -3,    /* workspace too small or misaligned */
+    HSTU_ERR_CUDA = -4          /* a CUDA runtime/driver call failed */
+} hstu_status_code;
+
+typedef enum { HSTU_DTYPE_BF16 = 0, HSTU_DTYPE_FP32 = 1 } hstu_dtype;
+
+/* Bits of the device status word (hstu_read_status). */
+enum {
+    HSTU_DEV_BAD_PAGE = 1u << 0,     /* page_table entry outside [0, num_pages) */
+    HSTU_DEV_BAD_LENGTH = 1u << 1,   /* negative length, num_targets > length, a cached or
+                                        appended position beyond max_pages_per_user * P,
+                                        or a length above the bound passed on the host */
+    HSTU_DEV_BAD_NMAX = 1u << 2,     /* a user's total length exceeds n_max */
+    HSTU_DEV_TIMEOUT = 1u << 3,      /* an in-kernel wait gave up (kernel returned early) */
+    HSTU_DEV_SMEM_ALIGN = 1u << 4    /* shared memory not aligned as the kernel requires */
+};
+
+typedef struct {
+    int32_t num_heads;            /* H >= 1 */
+    int32_t head_dim;             /* D in {32, 64, 128} */
+    int32_t dtype;                /* hstu_dtype */
+    int32_t num_buckets;          /* NB in [1, 4096] */
+    int32_t n_max;                /* >= 1: the 1/n_max weight scale and the bucket range;
+                                     every user's total length must be <= n_max */
+    int32_t page_size;            /* P (paged calls): 8, 16, 32, 64 or 128 */
+    int32_t num_pages;            /* physical pages in the pool (paged calls) */
+    int32_t max_pages_per_user;   /* row stride of page_table (paged calls) */
+    float ln_eps;                 /* LayerNorm epsilon, e.g. 1e-5 */
+} hstu_attn_params;
+
+/* Library version string. */
+const char* hstu_version(void);
+
+/* Human-readable text for an hstu_status_code. */
+const char* hstu_error_string(int code);
+
+/*
+ * Workspace bytes needed by one call with at most `max_batch` users, `max_tokens` query
+ * tokens in total (jagged: all tokens; paged: all new tokens) and at most `max_new`
+ * query tokens per user.  The same workspace serves jagged, paged and append calls whose
+ * sizes stay within those bounds.  Returns 0 for invalid params.
+ */
+size_t hstu_workspace_size(const hstu_attn_params* params, int32_t max_batch, int64_t max_tokens,
+                           int32_t max_new);
+
+/* Zero the workspace's status word (and nothing else needs zeroing).  Async on stream. */
+int hstu_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, copy the workspace's device status word to *flags_out (a bitwise
+ * OR of HSTU_DEV_* since the last clear) and, when `clear` is nonzero, reset it to 0.
+ */
+int hstu_read_status(void* workspace, void* stream, uint32_t* flags_out, int clear);
+
+/*
+ * Jagged prefill (no cache): every token of every user is a query.
+ *   q, k, v, u, out : [total_tokens][H][D]
+ *   seq_offsets     : [B+1] int32, seq_offsets[0] = 0, nondecreasing, seq_offsets[B] =
+ *                     total_tokens; user b owns rows seq_offsets[b] .. seq_offsets[b+1]-1
+ *   num_targets     : [B] int32 candidates at the end of each user's sequence, or NULL (0)
+ *   rab             : [H][NB] fp32
+ *   max_seqlen      : host-side upper bound on every user's length (sizes the grid; a user
+ *                     longer than it sets HSTU_DEV_BAD_LENGTH)
+ * Sections cited above: the HSTU attention formula; jagged inputs.
+ */
+int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const void* k,
+                         const void* v, const void* u, const int32_t* seq_offsets,
+                         const int32_t* num_targets, const float* rab, void* out, int32_t B,
+                         int64_t total_tokens, int32_t max_seqlen, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * Paged cache hit: only the new tokens of each user are queries.  User b's keys are its
+ * cached_lens[b] history tokens, read through page_table[b] (logical position p lives in
+ * page page_table[b][p / P], slot p % P), followed by its new_lens[b] new tokens.  New
+ * tokens of user b are rows off_b .. off_b + new_lens[b] - 1 of q_new/k_new/v_new/u_new/out,
+ * where off_b = new_lens[0] + ... + new_lens[b-1].  The last num_targets[b] new tokens are
+ * candidates.  New token t of user b sits at absolute position cached_lens[b] + t.
+ *   k_pages, v_pages : [num_pages][H][P][D]
+ *   page_table       : [B][max_pages_per_user] int32 (entries past the user's cached length
+ *                      are not read)
+ *   cached_lens, new_lens : [B] int32;  num_targets : [B] int32 or NULL (0)
+ *   total_new        : sum of new_lens (host value; sizes the epilogue)
+ *   max_new          : host-side upper bound on new_lens[b]
+ * The result does not depend on whether hstu_kv_append of these new tokens ran before.
+ * Sources: the paged GPU KV table and "compute only the new tokens" (NVIDIA blog, sections
+ * "Why serving large sequential recommenders is hard" and "Benefits").
+ */
+int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const void* k_new,
+                        const void* v_new, const void* u_new, const void* k_pages,
+                        const void* v_pages, const int32_t* page_table,
+                        const int32_t* cached_lens, const int32_t* new_lens,
+                        const int32_t* num_targets, const float* rab, void* out, int32_t B,
+                        int64_t total_new, int32_t max_new, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * Append new history tokens into the pages (the KV cache's "append"; NVIDIA blog, section
+ * "Why serving large sequential recommenders is hard").  For user b the first
+ * new_lens[b] - num_targets[b] rows of its new tokens (rows off_b.. of k_new/v_new, off_b
+ * as in hstu_attn_paged_fwd) are copied to logical positions cached_lens[b] + t; candidates
+ * are never appended.  A raw, bit-exact copy of K and V rows.  cached_lens is not modified:
+ * the caller advances it afterwards.
+ *   k_pages, v_pages : [num_pages][H][P][D], written
+ *   k_new, v_new     : [total_new][H][D]; a user whose rows would pass total_new is skipped
+ *                      and flagged (HSTU_DEV_BAD_LENGTH)
+ *   max_new          : host-side upper bound on new_lens[b]
+ * Tokens whose page id is invalid or whose position is beyond max_pages_per_user * P are
+ * skipped and flagged (HSTU_DEV_BAD_PAGE / HSTU_DEV_BAD_LENGTH).  The workspace is used
+ * only for that status word.
+ */
+int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages,
+                   const int32_t* page_table, const void* k_new, const void* v_new,
+                   const int32_t* cached_lens, const int32_t* new_lens,
+                   const int32_t* num_targets, int32_t B, int64_t total_new, int32_t max_new,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The library's own bucket table: table_out[d] = bucket(d) for d in [0, n), computed on the
+ * device in double precision (the function that the attention kernels use).  table_out is
+ * a device int32 array of n entries.  Exposed so that tests can compare it with an
+ * independent implementation.
+ */
+int hstu_bucket_table(const hstu_attn_params* params, int32_t n, int32_t* table_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_B200_H */

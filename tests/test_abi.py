@@ -1,0 +1,102 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol include/hstu.h
+declares, and rejects bad host-side arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hstu_attention_b200 as hb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hstu.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hstu_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hstu_attention_b200 import build
+
+    build.build()
+    return hb.load()
+
+
+def test_header_declares_the_api():
+    names = _declared()
+    assert "hstu_attn_jagged_fwd" in names and "hstu_attn_paged_fwd" in names and "hstu_kv_append" in names
+    assert set(names) == set(hb.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_error_strings(lib):
+    assert "sm_100a" in hb.version()
+    for code, text in [(0, "ok"), (-1, "invalid"), (-2, "unsupported"), (-3, "workspace"), (-4, "CUDA")]:
+        assert text in lib.hstu_error_string(code).decode()
+
+
+def _p(**kw):
+    base = dict(num_heads=4, head_dim=128, dtype="bf16", num_buckets=128, n_max=4096, page_size=32,
+                num_pages=64, max_pages_per_user=8)
+    base.update(kw)
+    return hb.params(**base)
+
+
+def test_workspace_size(lib):
+    p = _p()
+    n = hb.workspace_size(p, 8, 1000, 256)
+    assert n % 256 == 0 and n >= 256 + 1000 * 4 * 128 * 4
+    assert lib.hstu_workspace_size(None, 1, 1, 1) == 0
+    bad = _p(head_dim=96)
+    assert lib.hstu_workspace_size(ctypes.byref(bad), 1, 1, 1) == 0
+
+
+def test_host_validation_without_gpu(lib):
+    """Every call here fails host-side validation, so nothing reaches the device."""
+    p = _p()
+    fake = 1 << 20                      # aligned, never dereferenced
+    ws = 1 << 24
+    J = lib.hstu_attn_jagged_fwd
+    args = [fake, fake, fake, fake, fake, None, fake, fake, 2, 100, 64, ws, 1 << 30, None]
+    assert J(None, *args) == -1                                          # INVALID_ARG
+    assert J(ctypes.byref(_p(head_dim=96)), *args) == -2                  # UNSUPPORTED
+    assert J(ctypes.byref(_p(dtype="fp32", num_buckets=0)), *args) == -1
+    mis = list(args)
+    mis[0] = fake + 2                                                     # misaligned q
+    assert J(ctypes.byref(p), *mis) == -1
+    small = list(args)
+    small[-2] = 100                                                       # workspace too small
+    assert J(ctypes.byref(p), *small) == -3
+    unal = list(args)
+    unal[-3] = ws + 8                                                     # misaligned workspace
+    assert J(ctypes.byref(p), *unal) == -3
+    neg = list(args)
+    neg[8] = -1
+    assert J(ctypes.byref(p), *neg) == -1
+    # empty batch is a no-op success
+    empty = list(args)
+    empty[8] = 0
+    assert J(ctypes.byref(p), *empty) == 0
+
+    P = lib.hstu_attn_paged_fwd
+    pargs = [fake] * 6 + [fake, fake, fake, None, fake, fake, 2, 100, 64, ws, 1 << 30, None]
+    assert P(ctypes.byref(_p(page_size=24)), *pargs) == -2
+    assert P(ctypes.byref(_p(num_pages=0)), *pargs) == -1
+    nul = list(pargs)
+    nul[6] = None                                                         # page_table
+    assert P(ctypes.byref(p), *nul) == -1
+
+    A = lib.hstu_kv_append
+    aargs = [fake, fake, fake, fake, fake, fake, fake, None, 2, 100, 64, ws, 1 << 20, None]
+    assert A(ctypes.byref(_p(page_size=12)), *aargs) == -2
+    bad_ws = list(aargs)
+    bad_ws[-3] = None
+    assert A(ctypes.byref(p), *bad_ws) == -3
+    assert lib.hstu_bucket_table(ctypes.byref(p), -1, None, None) == -1
