@@ -50,7 +50,8 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+    """Samples nvidia-smi SM clocks and throttle reasons (every 100 ms, into a file) while the
+    timed region runs."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -58,25 +59,18 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.index = index
-        self.rows = []
         self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+                                          "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
         return self
-
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -87,18 +81,35 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except OSError:
+            pass
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [v for v in (num(r[1]) for r in rows) if v is not None]
+        mx = [v for v in (num(r[2]) for r in rows) if v is not None]
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = set()
-        for r in self.rows:
+        for r in rows:
             for name, val in zip(names, r[5:9]):
                 if val.strip().lower() == "active":
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(self.rows)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "window": "timed steps plus >= 0.3 s of identical graph replays before and after"}
 
 
 # ----------------------------------------------------------------------------- workload
@@ -313,17 +324,26 @@ def main():
     graph.replay()
     torch.cuda.synchronize()
 
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     call_ms = []
+    def roll(seconds):
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(20):
+                graph.replay()
+            torch.cuda.synchronize()
+
     with ClockSampler(local_rank) as clk:
+        roll(0.3)                      # clocks are sampled every 100 ms: keep the GPU busy around
+        if world > 1:                  # the timed window so samples land while it runs
+            dist.barrier()
+        torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(args.steps):
             graph.replay()
         e1.record(stream)
         torch.cuda.synchronize()
+        roll(0.3)
     elapsed_ms = e0.elapsed_time(e1)
     # per-call durations of the last replay's paged attention calls
     for a, b in events:

@@ -52,7 +52,11 @@ static int check_params(const hstu_attn_params* p, bool paged)
 
 static int esize_of(const hstu_attn_params* p) { return p->dtype == HSTU_DTYPE_FP32 ? 4 : 2; }
 
-static bool use_tc(const hstu_attn_params* p) { return p->dtype == HSTU_DTYPE_BF16 && p->head_dim == 128; }
+// The tensor-core kernel handles bf16, head_dim 128 and up to 1024 buckets (staged in shared memory).
+static bool use_tc(const hstu_attn_params* p)
+{
+    return p->dtype == HSTU_DTYPE_BF16 && p->head_dim == 128 && p->num_buckets <= 1024;
+}
 
 static int num_sms()
 {

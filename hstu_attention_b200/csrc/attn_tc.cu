@@ -3,7 +3,7 @@
 // What it computes (per user b, head h): for a block of 128 query rows and the key tiles the
 // block may see,
 //     S = Q K^T                               tcgen05.mma, accumulator in tensor memory
-//     P = allowed ? SiLU(S + rab[h][bucket(i-j)]) / n_max : 0      (registers, -> bf16)
+//     P = allowed ? SiLU(S + rab[h][bucket(i-j)]) : 0      (registers, -> bf16; 1/n_max on O)
 //     O += P V                                tcgen05.mma, accumulator in tensor memory
 // SiLU weighting replaces softmax, so there is no running max or row sum and key tiles can be
 // split across CTAs and summed afterwards (aitrends.kr summary, section "HSTU의 순차 모델링";
@@ -15,17 +15,24 @@
 //
 // CTA roles (384 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring.  Paged tiles
-//               are gathered page by page (one TMA box of P rows per page and channel half).
+//               are gathered page by page (one TMA box of P rows per page and channel half)
+//               using the page ids that warps 2-3 staged in shared memory.
 //   warp 1      allocates 512 TMEM columns; lane 0 issues all MMAs:
 //               S_t = Q K_t^T into S buffer t%2, then O += P_{t-1} V_{t-1}, so the pointwise
 //               work on S_t overlaps the P V product of the previous tile.
+//   warps 2-3   bias producers: for every tile they write the 255 distinct values
+//               rab[h][bucket(i-j)] / 2 the tile needs (i-j spans 255 values) into a
+//               double-buffered window, in four copies shifted by one float so that each
+//               pointwise thread reads its 64 values with 16-byte loads.
 //   warps 4-11  two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
 //               warp w%4 owns TMEM lanes (= query rows) [32(w%4), +32).  They load S from
-//               TMEM, add the bias, mask, apply SiLU/n_max, write bf16 P into shared memory in
-//               the 128-byte-swizzled K-major layout the MMA reads, and at the end move O
-//               from TMEM to the workspace.
-// Shared memory (1024-byte aligned, 128B swizzle everywhere):
-//   Q 32 KB | 2 x (K 32 KB + V 32 KB) | P 32 KB | 2 bias windows | mbarriers
+//               TMEM, form x/2 = S/2 + rab/2 with packed fp32x2 FMAs, mask, and write
+//               SiLU(x) = x/2 * (1 + tanh(x/2)) as bf16 P into shared memory in the
+//               128-byte-swizzled K-major layout the MMA reads.  The 1/n_max scale is applied
+//               once to O when it leaves TMEM.
+// Shared memory (1024-byte aligned, 128B swizzle for every MMA operand):
+//   Q 32 KB | 2 x (K 32 KB + V 32 KB) | P 32 KB | 2 bias windows | bucket bounds | rab |
+//   page ids | mbarriers
 // Every wait is bounded (HSTU_DEV_TIMEOUT) so a logic error cannot hang the GPU.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -38,15 +45,21 @@ constexpr int kTcD = 128;
 constexpr int kTile = 128;                    // query rows per CTA and keys per tile
 constexpr int kStages = 2;
 constexpr int kTcThreads = 384;
+constexpr int kMaxNB = 1024;                  // buckets staged in shared memory
+constexpr int kMaxPageIds = 1024;             // page ids staged per CTA (rest read from global)
 constexpr uint32_t kHalf = 128 * 128;         // 128 rows x 128 bytes = 16 KB (one swizzle column)
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffStage = 2 * kHalf;     // stage s at kOffStage + s * kStageBytes
 constexpr uint32_t kStageBytes = 4 * kHalf;   // K halves then V halves
 constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kWinStride = 260;          // floats per shifted copy (256 + 4: spreads banks)
+constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
 constexpr uint32_t kOffWin = kOffP + 2 * kHalf;
-constexpr uint32_t kWinFloats = 256;
-constexpr uint32_t kOffBar = kOffWin + 2 * kWinFloats * 4;
-constexpr int kNumBars = 14;
+constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
+constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
+constexpr uint32_t kOffPages = kOffRab + kMaxNB * 4;
+constexpr uint32_t kOffBar = kOffPages + kMaxPageIds * 4;
+constexpr int kNumBars = 18;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;     // slack to align the base to 1024
@@ -54,6 +67,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 
 struct TileGeo {
     int32_t j0;       // absolute position of key row 0 of the tile
@@ -76,6 +90,40 @@ __device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t ct, int32_t C, in
     return g;
 }
 
+// bucket(d) from the staged bounds: the largest k with bounds[k] <= d (bounds[nb] is a sentinel).
+__device__ __forceinline__ int bucket_from_bounds(const int32_t* bounds, int nb, int32_t d)
+{
+    int lo = 0, hi = nb;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (bounds[mid] <= d)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Smallest d >= 0 with bucket(d) >= k (bucket() of common.cuh, double precision), k >= 1.
+__device__ int bucket_bound(int k, double ln_nmax, int nb, int32_t n_max)
+{
+    if (nb <= 1 || !(ln_nmax > 0.0))
+        return 0x7fffffff;
+    if (k == 1)
+        return 1;
+    // bucket(d) >= k  <=>  (nb-1) ln d / ln n_max >= k-1; start at the real root, then fix up
+    // against the exact double evaluation so that both agree on every d.
+    double root = exp((double)(k - 1) * ln_nmax / (double)(nb - 1));
+    int64_t c = (int64_t)ceil(root);
+    if (c < 1)
+        c = 1;
+    for (int it = 0; it < 8 && c > 1 && bucket_of(c - 1, ln_nmax, nb) >= k; ++it)
+        --c;
+    for (int it = 0; it < 8 && bucket_of(c, ln_nmax, nb) < k; ++it)
+        ++c;
+    return c > 0x7ffffffe ? 0x7ffffffe : (int)c;
+}
+
 template <bool kPaged>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -86,15 +134,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ UserGeom sG;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.z, h = blockIdx.y;
+    // grid: x = (split, head, user) fastest-varying, y = query block, heaviest blocks first
     const int split = blockIdx.x % a.splits;
-    const int qblk = a.qblocks - 1 - (int)(blockIdx.x / a.splits);     // heaviest query blocks first
+    const int h = (blockIdx.x / a.splits) % a.H;
+    const int b = blockIdx.x / (a.splits * a.H);
+    const int qblk = a.qblocks - 1 - (int)blockIdx.y;
 
     if (warp == 0) {
+        const bool report = qblk == 0 && h == 0 && split == 0;
         UserGeom g = kPaged ? paged_geom(a.cached_lens, a.new_lens, a.num_targets, b, a.total_tokens, a.max_len,
-                                         a.max_pages * a.P, a.n_max, a.ws, blockIdx.x == 0 && h == 0)
+                                         a.max_pages * a.P, a.n_max, a.ws, report)
                             : jagged_geom(a.seq_offsets, a.num_targets, b, a.total_tokens, a.max_len, a.n_max,
-                                          a.ws, blockIdx.x == 0 && h == 0);
+                                          a.ws, report);
         if (lane == 0)
             sG = g;
     }
@@ -142,9 +193,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* p_full = bars + 11;
     uint64_t* p_empty = bars + 12;
     uint64_t* o_full = bars + 13;
+    uint64_t* win_full = bars + 14;   // [2]
+    uint64_t* win_empty = bars + 16;  // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* win = reinterpret_cast<float*>(smem + kOffWin);
+    int32_t* s_bounds = reinterpret_cast<int32_t*>(smem + kOffBounds);
+    float* s_rab = reinterpret_cast<float*>(smem + kOffRab);
+    int32_t* s_pages = reinterpret_cast<int32_t*>(smem + kOffPages);
+
+    // cached logical pages this CTA reads: [lp_begin, lp_end)
+    const int P = kPaged ? a.P : 1;
+    const int32_t lp_begin = kPaged ? (t_begin < ct ? t_begin * (kTile / P) : 0) : 0;
+    const int32_t lp_end = kPaged ? (t_begin < ct ? min(min(t_end, ct) * (kTile / P), (g.C + P - 1) / P) : 0) : 0;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -156,6 +217,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], 256);
+            mbar_init(&win_full[s], 64);
+            mbar_init(&win_empty[s], 256);
         }
         mbar_init(p_full, 256);
         mbar_init(p_empty, 1);
@@ -166,6 +229,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
+    }
+    if (kPaged && (warp == 2 || warp == 3)) {
+        // stage this CTA's page ids (validated; -1 = skip the load)
+        for (int k = threadIdx.x - 64; k < lp_end - lp_begin && k < kMaxPageIds; k += 64) {
+            int32_t pg = a.page_table[(int64_t)b * a.max_pages + lp_begin + k];
+            if (pg < 0 || pg >= a.num_pages) {
+                set_flag(a.ws, HSTU_DEV_BAD_PAGE);
+                pg = -1;
+            }
+            s_pages[k] = pg;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -195,7 +269,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t kdst = sbase + kOffStage + st * kStageBytes;
             const uint32_t vdst = kdst + 2 * kHalf;
             if (kPaged && tg.cached) {
-                const int P = a.P;
                 const int lp0 = tg.j0 / P;
                 const int npg = kTile / P;
                 uint32_t bytes = 0;
@@ -203,14 +276,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int k = 0; k < npg; ++k) {
                     const int lp = lp0 + k;
                     int32_t pg = -1;
-                    if (lp * P < g.C) {
-                        pg = a.page_table[(int64_t)b * a.max_pages + lp];
-                        if (pg < 0 || pg >= a.num_pages) {
-                            set_flag(a.ws, HSTU_DEV_BAD_PAGE);
-                            pg = -1;
+                    if (lp < lp_end) {
+                        const int idx = lp - lp_begin;
+                        if (idx < kMaxPageIds) {
+                            pg = s_pages[idx];
                         } else {
-                            bytes += (uint32_t)P * 128u * 2u;
+                            pg = a.page_table[(int64_t)b * a.max_pages + lp];
+                            if (pg < 0 || pg >= a.num_pages) {
+                                set_flag(a.ws, HSTU_DEV_BAD_PAGE);
+                                pg = -1;
+                            }
                         }
+                        if (pg >= 0)
+                            bytes += (uint32_t)P * 128u * 2u;
                     }
                     pages[k] = pg;
                 }
@@ -311,72 +389,117 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         umma_commit(o_full);
         volatile int never = 0;
         mbar_wait(o_full, 0, &never, tmo);
+    } else if (warp == 2 || warp == 3) {
+        // ============================================================ bias window producers
+        const int ht = threadIdx.x - 64;                  // 0..63
+        named_barrier_sync(2, 320);                       // bounds and rab staged by warps 4-11
+        const int nb = a.NB;
+        bool ok = true;
+        for (int t = 0; t < n; ++t) {
+            const int wb = t & 1;
+            if (t >= 2) {
+                ok = ok && mbar_wait(&win_empty[wb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
+                if (!ok)
+                    break;
+            }
+            const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
+            const int32_t dist0 = i0 - tg.j0 + (kTile - 1);       // distance at window index 0
+            float* wbuf = win + wb * (kWinBuf / 4);
+            for (int y = ht; y < 256; y += 64) {
+                const int32_t d = dist0 - y;
+                const float val = (y <= 2 * kTile - 2 && d >= 0) ? 0.5f * s_rab[bucket_from_bounds(s_bounds, nb, d)]
+                                                                 : 0.f;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    if (y - s >= 0)
+                        wbuf[s * kWinStride + (y - s)] = val;
+            }
+            mbar_arrive(&win_full[wb]);
+        }
     } else if (warp >= 4) {
         // ============================================================ pointwise + epilogue
         const int pt = threadIdx.x - 128;                 // 0..255
+        // stage rab[h][:] and the bucket bounds, then release the bias producers
+        for (int k = pt; k < a.NB; k += 256)
+            s_rab[k] = a.rab[(int64_t)h * a.NB + k];
+        for (int k = pt; k <= a.NB; k += 256)
+            s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB, a.n_max));
+        named_barrier_sync(2, 320);
+
         const int wg = (warp - 4) >> 2;                   // key-column half
         const int r = ((warp & 3) << 5) + lane;           // query row in the block (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const bool row_valid = qrow0 + r < g.N;
         const int32_t i_abs = i0 + r;
         const int32_t lim_row = row_valid ? min(i_abs + 1, g.hist) : -1;
-        const float half_inv_n = 0.5f * a.inv_n;
-        const float* rab_h = a.rab + (int64_t)h * a.NB;
+        // window: this thread's 64 bias values start at index y0 = 127 - r + 64 wg; copy s holds
+        // the window shifted by s floats, so (y0 - s) is a multiple of 4
+        const int y0 = (kTile - 1) - r + 64 * wg;
+        const int wsel = y0 & 3;
+        const int woff = wsel * kWinStride + (y0 - wsel);
         uint8_t* pbuf = smem + kOffP + wg * kHalf + r * 128;
+        const uint64_t half2 = f2pack(0.5f, 0.5f);
         bool ok = true;
         for (int t = 0; t < n; ++t) {
             const int st = t % kStages;
             const uint32_t kph = (t / kStages) & 1;
             const int sb = t & 1;
             const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
-            float* w_t = win + sb * kWinFloats;
-            if (pt < 2 * kTile - 1) {
-                const int64_t dist = (int64_t)i0 - tg.j0 - (kTile - 1) + pt;
-                w_t[pt] = dist >= 0 ? rab_h[bucket_of(dist, a.ln_nmax, a.NB)] : 0.f;
-            }
-            named_barrier_sync(1, 256);
             ok = ok && mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
+            ok = ok && mbar_wait(&win_full[sb], (t >> 1) & 1, abort_flag, tmo);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
-                continue;
+                break;
             tc_fence_after();
-            uint32_t sv[2][32];
+            uint32_t sv[64];
             const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0) + wg * 64;
-            tmem_ld_32x32b_x32(scol, sv[0]);
-            tmem_ld_32x32b_x32(scol + 32, sv[1]);
+            tmem_ld_32x32b_x32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld_32x32b_x32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_empty[sb]);
 
+            const float4* wv = reinterpret_cast<const float4*>(win + sb * (kWinBuf / 4) + woff);
             const bool full = (qrow0 + kTile - 1 < g.N) && (tg.j0 + kTile - 1 < tg.kvend) &&
                               (tg.j0 + kTile - 1 <= i0) && (tg.j0 + kTile - 1 < g.hist);
             const int32_t lim = min(lim_row, tg.kvend);
             const int32_t diag = (row_valid && !tg.cached) ? i_abs : -1;
             const int jc0 = tg.j0 + wg * 64;                  // key position of column 0 of this half
-            const float* wrow = w_t + r + (kTile - 1) - wg * 64;   // wrow[-c] = bias at column c
             uint32_t packed[32];
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-                // SiLU(x) / n_max = hx * (1 + tanh(x / 2)) with hx = x / (2 n_max)
-                const float x0 = __uint_as_float(sv[c >> 5][c & 31]) + wrow[-c];
-                const float x1 = __uint_as_float(sv[(c + 1) >> 5][(c + 1) & 31]) + wrow[-(c + 1)];
-                const float h0 = x0 * half_inv_n, h1 = x1 * half_inv_n;
-                float w0 = fmaf(h0, tanh_approx(0.5f * x0), h0);
-                float w1 = fmaf(h1, tanh_approx(0.5f * x1), h1);
+            for (int q4 = 0; q4 < 16; ++q4) {
+                const float4 bias = wv[q4];
+                // x/2 = S/2 + rab/2 for four columns, as two packed pairs
+                const uint64_t xa = f2fma(f2pack(__uint_as_float(sv[4 * q4]), __uint_as_float(sv[4 * q4 + 1])), half2,
+                                          f2pack(bias.x, bias.y));
+                const uint64_t xb = f2fma(f2pack(__uint_as_float(sv[4 * q4 + 2]), __uint_as_float(sv[4 * q4 + 3])),
+                                          half2, f2pack(bias.z, bias.w));
+                float a0, a1, a2, a3;
+                f2unpack(xa, a0, a1);
+                f2unpack(xb, a2, a3);
+                // SiLU(x) = x/2 * (1 + tanh(x/2))
+                const uint64_t wa = f2fma(xa, f2pack(tanh_approx(a0), tanh_approx(a1)), xa);
+                const uint64_t wb2 = f2fma(xb, f2pack(tanh_approx(a2), tanh_approx(a3)), xb);
+                float w0, w1, w2, w3;
+                f2unpack(wa, w0, w1);
+                f2unpack(wb2, w2, w3);
                 if (!full) {
-                    const int j = jc0 + c;
+                    const int j = jc0 + 4 * q4;
                     w0 = ((j < lim) || (j == diag)) ? w0 : 0.f;
                     w1 = ((j + 1 < lim) || (j + 1 == diag)) ? w1 : 0.f;
+                    w2 = ((j + 2 < lim) || (j + 2 == diag)) ? w2 : 0.f;
+                    w3 = ((j + 3 < lim) || (j + 3 == diag)) ? w3 : 0.f;
                 }
-                __nv_bfloat162 p2 = __floats2bfloat162_rn(w0, w1);
-                packed[c >> 1] = *reinterpret_cast<uint32_t*>(&p2);
+                packed[2 * q4] = bf16x2_rn(w0, w1);
+                packed[2 * q4 + 1] = bf16x2_rn(w2, w3);
             }
+            mbar_arrive(&win_empty[sb]);
             if (t >= 1) {
                 ok = ok && mbar_wait(p_empty, (t - 1) & 1, abort_flag, tmo);
                 ok = __all_sync(0xffffffffu, ok);
+                if (!ok)
+                    break;
             }
-            if (!ok)
-                continue;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 uint4 v4 = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
@@ -400,25 +523,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 mbar_arrive(p_full);
             }
         }
-        // ------------------------------------------------------------ epilogue: O -> workspace
+        // ------------------------------------------------------------ epilogue: O / n_max -> workspace
         ok = ok && mbar_wait(o_full, 0, abort_flag, tmo);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc_fence_after();
-            uint32_t ov[2][32];
+            uint32_t ov[64];
             const uint32_t ocol = tmem + lane_base + kColO + wg * 64;
-            tmem_ld_32x32b_x32(ocol, ov[0]);
-            tmem_ld_32x32b_x32(ocol + 32, ov[1]);
+            tmem_ld_32x32b_x32(ocol, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+            tmem_ld_32x32b_x32(ocol + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
             tmem_wait_ld();
             if (row_valid) {
+                const float inv_n = a.inv_n;
                 float4* dst = reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + r) * HD + (int64_t)h * kTcD + wg * 64);
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4) {
-                    const int c = c4 * 4;
-                    dst[c4] = make_float4(__uint_as_float(ov[c >> 5][c & 31]), __uint_as_float(ov[c >> 5][(c & 31) + 1]),
-                                          __uint_as_float(ov[c >> 5][(c & 31) + 2]),
-                                          __uint_as_float(ov[c >> 5][(c & 31) + 3]));
-                }
+                for (int c4 = 0; c4 < 16; ++c4)
+                    dst[c4] = make_float4(__uint_as_float(ov[4 * c4]) * inv_n, __uint_as_float(ov[4 * c4 + 1]) * inv_n,
+                                          __uint_as_float(ov[4 * c4 + 2]) * inv_n,
+                                          __uint_as_float(ov[4 * c4 + 3]) * inv_n);
             }
         }
     }
@@ -439,10 +561,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 void launch_attn_tc(const TcMaps& m, const TcArgs& a, bool paged, int32_t B, cudaStream_t stream)
 {
     static bool attr_set[2] = {false, false};
-    const int grid_x = a.qblocks * a.splits;
-    if (B <= 0 || grid_x <= 0)
+    const int64_t grid_x = (int64_t)a.splits * a.H * B;
+    if (B <= 0 || grid_x <= 0 || a.qblocks <= 0)
         return;
-    dim3 grid(grid_x, a.H, B);
+    dim3 grid((unsigned)grid_x, (unsigned)a.qblocks, 1);
     if (paged) {
         if (!attr_set[1]) {
             cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
