@@ -3,19 +3,88 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
+#include <map>
 #include <mutex>
 #include <stdint.h>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace hstu {
 
-__global__ void bucket_table_kernel(int32_t n, double ln_nmax, int32_t nb, int32_t* out)
+__global__ void bucket_table_kernel(int32_t n, double ln_nmax, int32_t nb, const __grid_constant__ BucketBounds bb,
+                                    int32_t* out)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n)
+    if (i >= n)
+        return;
+    if (bb.count > 0) {
+        // the largest k with v[k] <= i: the same table the tensor-core kernels use
+        int lo = 0, hi = bb.count - 1;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (bb.v[mid] <= i)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        out[i] = lo;
+    } else {
         out[i] = bucket_of(i, ln_nmax, nb);
+    }
+}
+
+// bucket(d) evaluated on the host in double precision (the library's definition).
+static int host_bucket(int64_t d, double ln_nmax, int nb)
+{
+    if (nb <= 1 || d <= 0 || !(ln_nmax > 0.0))
+        return 0;
+    const double x = (double)(nb - 1) * log((double)d) / ln_nmax;
+    const int64_t b = 1 + (int64_t)floor(x);
+    return (int)(b > nb - 1 ? nb - 1 : b);
+}
+
+// Boundaries of the log-spaced buckets for (n_max, nb), cached per pair (a few hundred bytes).
+static BucketBounds host_bounds(int32_t n_max, int32_t nb)
+{
+    static std::mutex mu;
+    static std::map<std::pair<int32_t, int32_t>, BucketBounds> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(n_max, nb);
+    auto it = cache.find(key);
+    if (it != cache.end())
+        return it->second;
+    BucketBounds bb{};
+    if (nb > kMaxParamNB) {
+        bb.count = 0;
+    } else {
+        const double ln_nmax = log((double)n_max);
+        bb.count = nb + 1;
+        bb.v[0] = 0;
+        for (int k = 1; k < nb; ++k) {
+            int64_t c;
+            if (nb <= 1 || !(ln_nmax > 0.0)) {
+                c = 0x7fffffff;
+            } else if (k == 1) {
+                c = 1;
+            } else {
+                c = (int64_t)ceil(exp((double)(k - 1) * ln_nmax / (double)(nb - 1)));
+                if (c < 1)
+                    c = 1;
+                while (c > 1 && host_bucket(c - 1, ln_nmax, nb) >= k)
+                    --c;
+                while (host_bucket(c, ln_nmax, nb) < k && c < 0x7fffffff)
+                    ++c;
+            }
+            bb.v[k] = (int32_t)(c > 0x7fffffff ? 0x7fffffff : c);
+        }
+        bb.v[nb] = 0x7fffffff;
+    }
+    if (cache.size() > 64)
+        cache.clear();
+    cache[key] = bb;
+    return bb;
 }
 
 // ------------------------------------------------------------------ helpers
@@ -209,8 +278,9 @@ int hstu_bucket_table(const hstu_attn_params* params, int32_t n, int32_t* table_
     if (n == 0)
         return HSTU_OK;
     const double ln_nmax = log((double)params->n_max);
-    bucket_table_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(n, ln_nmax,
-                                                                                        params->num_buckets, table_out);
+    const BucketBounds bb = host_bounds(params->n_max, params->num_buckets);
+    bucket_table_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        n, ln_nmax, params->num_buckets, bb, table_out);
     return finish(static_cast<cudaStream_t>(stream));
 }
 
@@ -287,7 +357,7 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.timeout_ns = kTimeoutNs;
-        launch_attn_tc(m, a, false, B, s);
+        launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), false, B, s);
     } else {
         SimtArgs a{};
         a.q = q;
@@ -373,7 +443,7 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.timeout_ns = kTimeoutNs;
-        launch_attn_tc(m, a, true, B, s);
+        launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), true, B, s);
     } else {
         SimtArgs a{};
         a.q = q_new;

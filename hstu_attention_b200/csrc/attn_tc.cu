@@ -2,37 +2,39 @@
 //
 // What it computes (per user b, head h): for a block of 128 query rows and the key tiles the
 // block may see,
-//     S = Q K^T                               tcgen05.mma, accumulator in tensor memory
-//     P = allowed ? SiLU(S + rab[h][bucket(i-j)]) : 0      (registers, -> bf16; 1/n_max on O)
-//     O += P V                                tcgen05.mma, accumulator in tensor memory
+//     S = Q K^T                               tcgen05.mma (A, B in shared memory), S in TMEM
+//     P = allowed ? SiLU(S + rab[h][bucket(i-j)]) : 0      registers -> bf16 P in TMEM
+//     O += P V                                tcgen05.mma (A = P in TMEM, B = V in smem)
+//     O / n_max -> workspace (fp32)
 // SiLU weighting replaces softmax, so there is no running max or row sum and key tiles can be
 // split across CTAs and summed afterwards (aitrends.kr summary, section "HSTU의 순차 모델링";
 // news.bpdata.com, section "HSTU").  Keys of the paged layout come from the per-user page
 // table for positions below cached_len and from the new-token rows after that (NVIDIA blog
 // "Deploying an HSTU Generative Recommender with NVIDIA Dynamo-Triton", section "Why serving
 // large sequential recommenders is hard": the attention kernel reads K/V from the paged
-// cache).  O (fp32) goes to the workspace; combine.cu applies LayerNorm(O) * U.
+// cache).  combine.cu applies LayerNorm(O) * U to the fp32 partial outputs.
 //
 // CTA roles (384 threads):
-//   warp 0      TMA producer: Q once, then K and V tiles into a 2-stage ring.  Paged tiles
-//               are gathered page by page (one TMA box of P rows per page and channel half)
-//               using the page ids that warps 2-3 staged in shared memory.
-//   warp 1      allocates 512 TMEM columns; lane 0 issues all MMAs:
+//   warp 0      TMA producer of Q and of the K tiles (2-stage ring; a K stage frees as soon as
+//               Q K^T has read it).  Paged tiles are gathered page by page (one TMA box of P
+//               rows per page and channel half) using page ids staged in shared memory.
+//   warp 3      TMA producer of the V tiles (3-stage ring, freed after P V).
+//   warp 1      allocates all 512 TMEM columns; lane 0 issues every MMA:
 //               S_t = Q K_t^T into S buffer t%2, then O += P_{t-1} V_{t-1}, so the pointwise
 //               work on S_t overlaps the P V product of the previous tile.
-//   warps 2-3   bias producers: for every tile they write the 255 distinct values
-//               rab[h][bucket(i-j)] / 2 the tile needs (i-j spans 255 values) into a
-//               double-buffered window, in four copies shifted by one float so that each
-//               pointwise thread reads its 64 values with 16-byte loads.
+//   warp 2      bias producer: for every tile it writes the 255 distinct values
+//               rab[h][bucket(i-j)] / 2 the tile needs into a double-buffered window, in four
+//               copies shifted by one float so each pointwise thread reads 16-byte vectors.
 //   warps 4-11  two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
 //               warp w%4 owns TMEM lanes (= query rows) [32(w%4), +32).  They load S from
-//               TMEM, form x/2 = S/2 + rab/2 with packed fp32x2 FMAs, mask, and write
-//               SiLU(x) = x/2 * (1 + tanh(x/2)) as bf16 P into shared memory in the
-//               128-byte-swizzled K-major layout the MMA reads.  The 1/n_max scale is applied
-//               once to O when it leaves TMEM.
+//               TMEM, form x/2 = S/2 + rab/2 with packed fp32x2 FMAs, mask, compute
+//               SiLU(x) = x/2 * (1 + tanh(x/2)), and store it as bf16 P into TMEM (P buffer
+//               t%2), where the P V MMA reads it.  The 1/n_max scale is applied to O once,
+//               when it leaves TMEM.
+// TMEM columns: S0 [0,128) | S1 [128,256) | O [256,384) | P0 [384,448) | P1 [448,512)
 // Shared memory (1024-byte aligned, 128B swizzle for every MMA operand):
-//   Q 32 KB | 2 x (K 32 KB + V 32 KB) | P 32 KB | 2 bias windows | bucket bounds | rab |
-//   page ids | mbarriers
+//   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 2 bias windows | bucket bounds | rab | page ids |
+//   mbarriers
 // Every wait is bounded (HSTU_DEV_TIMEOUT) so a logic error cannot hang the GPU.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -43,28 +45,29 @@ using namespace sm100;
 
 constexpr int kTcD = 128;
 constexpr int kTile = 128;                    // query rows per CTA and keys per tile
-constexpr int kStages = 2;
+constexpr int kKStages = 2;
+constexpr int kVStages = 3;
 constexpr int kTcThreads = 384;
 constexpr int kMaxNB = 1024;                  // buckets staged in shared memory
 constexpr int kMaxPageIds = 1024;             // page ids staged per CTA (rest read from global)
 constexpr uint32_t kHalf = 128 * 128;         // 128 rows x 128 bytes = 16 KB (one swizzle column)
+constexpr uint32_t kTileBytes = 2 * kHalf;    // one 128 x 128 bf16 operand
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = 2 * kHalf;     // stage s at kOffStage + s * kStageBytes
-constexpr uint32_t kStageBytes = 4 * kHalf;   // K halves then V halves
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffK = kTileBytes;
+constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
 constexpr uint32_t kWinStride = 260;          // floats per shifted copy (256 + 4: spreads banks)
 constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
-constexpr uint32_t kOffWin = kOffP + 2 * kHalf;
+constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffPages = kOffRab + kMaxNB * 4;
 constexpr uint32_t kOffBar = kOffPages + kMaxPageIds * 4;
-constexpr int kNumBars = 18;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1 + 2 + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;     // slack to align the base to 1024
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
@@ -90,29 +93,68 @@ __device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t ct, int32_t C, in
     return g;
 }
 
-// bucket(d) from the staged bounds: the largest k with bounds[k] <= d (bounds[nb] is a sentinel).
-__device__ __forceinline__ int bucket_from_bounds(const int32_t* bounds, int nb, int32_t d)
+// bucket(d) from a float estimate of the log-spaced index, corrected against the exact
+// bounds (bounds[k] = smallest d with bucket(d) >= k, bounds[nb] a sentinel).  The estimate's
+// error is far below one bucket, so one step of correction suffices.
+// lg_scale = (nb - 1) / log2(n_max).
+__device__ __forceinline__ int bucket_fast(const int32_t* bounds, int nb, int32_t d, float lg_scale)
 {
-    int lo = 0, hi = nb;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (bounds[mid] <= d)
-            lo = mid;
-        else
-            hi = mid;
-    }
-    return lo;
+    if (d <= 0 || nb <= 1)
+        return 0;
+    int b = 1 + __float2int_rd(__log2f((float)d) * lg_scale);
+    b = max(1, min(b, nb - 1));
+    if (d < bounds[b])
+        --b;
+    else if (d >= bounds[b + 1])
+        ++b;
+    return b;
 }
 
-// Smallest d >= 0 with bucket(d) >= k (bucket() of common.cuh, double precision), k >= 1.
-__device__ int bucket_bound(int k, double ln_nmax, int nb, int32_t n_max)
+// SiLU weights of 32 consecutive key columns of one query row: x/2 = S/2 + bias (bias holds
+// rab/2), w = x/2 * (1 + tanh(x/2)), masked to 0 where the key is not visible, packed to
+// bf16x2.
+// kMasked selects the per-column visibility test at compile time, so the full-tile loop has
+// no branch and the compiler can interleave the independent tanh chains.
+template <bool kMasked>
+__device__ __forceinline__ void silu_cols32(const uint32_t* sv, const float4* wv, uint32_t* packed, int jc,
+                                            int32_t lim, int32_t diag)
+{
+    const uint64_t half2 = f2pack(0.5f, 0.5f);
+#pragma unroll
+    for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 bias = wv[q4];
+        const uint64_t xa = f2fma(f2pack(__uint_as_float(sv[4 * q4]), __uint_as_float(sv[4 * q4 + 1])), half2,
+                                  f2pack(bias.x, bias.y));
+        const uint64_t xb = f2fma(f2pack(__uint_as_float(sv[4 * q4 + 2]), __uint_as_float(sv[4 * q4 + 3])), half2,
+                                  f2pack(bias.z, bias.w));
+        float a0, a1, a2, a3;
+        f2unpack(xa, a0, a1);
+        f2unpack(xb, a2, a3);
+        const uint64_t wa = f2fma(xa, f2pack(tanh_approx(a0), tanh_approx(a1)), xa);
+        const uint64_t wb = f2fma(xb, f2pack(tanh_approx(a2), tanh_approx(a3)), xb);
+        float w0, w1, w2, w3;
+        f2unpack(wa, w0, w1);
+        f2unpack(wb, w2, w3);
+        if (kMasked) {
+            const int j = jc + 4 * q4;
+            w0 = ((j < lim) || (j == diag)) ? w0 : 0.f;
+            w1 = ((j + 1 < lim) || (j + 1 == diag)) ? w1 : 0.f;
+            w2 = ((j + 2 < lim) || (j + 2 == diag)) ? w2 : 0.f;
+            w3 = ((j + 3 < lim) || (j + 3 == diag)) ? w3 : 0.f;
+        }
+        packed[2 * q4] = bf16x2_rn(w0, w1);
+        packed[2 * q4 + 1] = bf16x2_rn(w2, w3);
+    }
+}
+
+// Smallest d >= 0 with bucket(d) >= k (bucket_of() of common.cuh, double precision), k >= 1.
+// Used when the host did not pass the bounds (more buckets than the parameter block holds).
+__device__ int bucket_bound(int k, double ln_nmax, int nb)
 {
     if (nb <= 1 || !(ln_nmax > 0.0))
         return 0x7fffffff;
     if (k == 1)
         return 1;
-    // bucket(d) >= k  <=>  (nb-1) ln d / ln n_max >= k-1; start at the real root, then fix up
-    // against the exact double evaluation so that both agree on every d.
     double root = exp((double)(k - 1) * ln_nmax / (double)(nb - 1));
     int64_t c = (int64_t)ceil(root);
     if (c < 1)
@@ -128,7 +170,8 @@ template <bool kPaged>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
-               const __grid_constant__ CUtensorMap tm_vp, const TcArgs a)
+               const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ BucketBounds bb,
+               const TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ UserGeom sG;
@@ -184,17 +227,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* smem = smem_raw + pad;
     const uint32_t sbase = raw_u32 + pad;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;      // [2]
-    uint64_t* v_full = bars + 3;      // [2]
-    uint64_t* kv_empty = bars + 5;    // [2]
-    uint64_t* s_full = bars + 7;      // [2]
-    uint64_t* s_empty = bars + 9;     // [2]
-    uint64_t* p_full = bars + 11;
-    uint64_t* p_empty = bars + 12;
-    uint64_t* o_full = bars + 13;
-    uint64_t* win_full = bars + 14;   // [2]
-    uint64_t* win_empty = bars + 16;  // [2]
+    uint64_t* q_full = bars;
+    uint64_t* k_full = q_full + 1;              // [kKStages]
+    uint64_t* k_empty = k_full + kKStages;      // [kKStages]
+    uint64_t* v_full = k_empty + kKStages;      // [kVStages]
+    uint64_t* v_empty = v_full + kVStages;      // [kVStages]
+    uint64_t* s_full = v_empty + kVStages;      // [2]
+    uint64_t* s_empty = s_full + 2;             // [2]
+    uint64_t* p_full = s_empty + 2;             // [2]
+    uint64_t* p_empty = p_full + 2;             // [2]
+    uint64_t* o_full = p_empty + 2;
+    uint64_t* win_full = o_full + 1;            // [2]
+    uint64_t* win_empty = win_full + 2;         // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* win = reinterpret_cast<float*>(smem + kOffWin);
@@ -209,19 +253,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kKStages; ++s) {
             mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
             mbar_init(&v_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], 256);
-            mbar_init(&win_full[s], 64);
+            mbar_init(&p_full[s], 256);
+            mbar_init(&p_empty[s], 1);
+            mbar_init(&win_full[s], 32);
             mbar_init(&win_empty[s], 256);
         }
-        mbar_init(p_full, 256);
-        mbar_init(p_empty, 1);
         mbar_init(o_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -230,16 +277,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (kPaged && (warp == 2 || warp == 3)) {
-        // stage this CTA's page ids (validated; -1 = skip the load)
-        for (int k = threadIdx.x - 64; k < lp_end - lp_begin && k < kMaxPageIds; k += 64) {
-            int32_t pg = a.page_table[(int64_t)b * a.max_pages + lp_begin + k];
-            if (pg < 0 || pg >= a.num_pages) {
-                set_flag(a.ws, HSTU_DEV_BAD_PAGE);
-                pg = -1;
+    if (warp == 2 || warp == 3) {
+        const int ht = threadIdx.x - 64;
+        if (kPaged) {
+            // this CTA's page ids (validated; -1 = skip the load)
+            for (int k = ht; k < lp_end - lp_begin && k < kMaxPageIds; k += 64) {
+                int32_t pg = a.page_table[(int64_t)b * a.max_pages + lp_begin + k];
+                if (pg < 0 || pg >= a.num_pages) {
+                    set_flag(a.ws, HSTU_DEV_BAD_PAGE);
+                    pg = -1;
+                }
+                s_pages[k] = pg;
             }
-            s_pages[k] = pg;
         }
+        for (int k = ht; k < a.NB; k += 64)
+            s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
+        if (bb.count > 0) {
+            for (int k = ht; k <= a.NB; k += 64)
+                s_bounds[k] = bb.v[k];
+        }
+    }
+    if (bb.count == 0 && warp >= 4) {
+        // bounds not passed by the host (many buckets): evaluate them here
+        for (int k = threadIdx.x - 128; k <= a.NB; k += 256)
+            s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB));
     }
     tc_fence_before();
     __syncthreads();
@@ -247,32 +308,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = a.timeout_ns;
 
-    if (warp == 0 && lane == 0) {
-        // ============================================================ TMA producer
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        if (kPaged) {
-            tma_prefetch_desc(&tm_kp);
-            tma_prefetch_desc(&tm_vp);
+    if ((warp == 0 || warp == 3) && lane == 0) {
+        // ============================================================ TMA producers
+        // warp 0 loads Q and the K tiles, warp 3 the V tiles: a single thread issuing every
+        // page box of a paged tile would serialise on TMA issue latency.
+        const bool is_v = warp == 3;
+        uint64_t* full = is_v ? v_full : k_full;
+        uint64_t* empty = is_v ? v_empty : k_empty;
+        const int stages = is_v ? kVStages : kKStages;
+        const uint32_t ring = sbase + (is_v ? kOffV : kOffK);
+        const CUtensorMap* tm_rows = is_v ? &tm_v : &tm_k;
+        const CUtensorMap* tm_pages = is_v ? &tm_vp : &tm_kp;
+        tma_prefetch_desc(tm_rows);
+        if (kPaged)
+            tma_prefetch_desc(tm_pages);
+        if (!is_v) {
+            tma_prefetch_desc(&tm_q);
+            mbar_arrive_expect_tx(q_full, kTileBytes);
+            for (int hf = 0; hf < 2; ++hf)
+                tma_load_3d(&tm_q, sbase + kOffQ + hf * kHalf, q_full, hf * 64, h, (int32_t)(g.tok0 + qrow0));
         }
-        mbar_arrive_expect_tx(q_full, 2 * kHalf);
-        for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(&tm_q, sbase + kOffQ + hf * kHalf, q_full, hf * 64, h, (int32_t)(g.tok0 + qrow0));
         int issued = 0;
         for (int t = 0; t < n; ++t) {
-            const int st = t % kStages;
-            const uint32_t kph = (t / kStages) & 1;
-            if (t >= kStages && !mbar_wait(&kv_empty[st], kph ^ 1, abort_flag, tmo))
-                break;
             const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
-            const uint32_t kdst = sbase + kOffStage + st * kStageBytes;
-            const uint32_t vdst = kdst + 2 * kHalf;
+            const int st = t % stages;
+            // tile t goes into stage t % stages once the MMA that read tile t - stages is done
+            if (t >= stages && !mbar_wait(&empty[st], ((t / stages) & 1) ^ 1, abort_flag, tmo))
+                break;
+            const uint32_t dst = ring + st * kTileBytes;
             if (kPaged && tg.cached) {
+                // gather: one box of P rows per cached page and channel half
                 const int lp0 = tg.j0 / P;
                 const int npg = kTile / P;
-                uint32_t bytes = 0;
                 int32_t pages[kTile / 8];
+                uint32_t bytes = 0;
                 for (int k = 0; k < npg; ++k) {
                     const int lp = lp0 + k;
                     int32_t pg = -1;
@@ -292,84 +361,65 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                     pages[k] = pg;
                 }
-                mbar_arrive_expect_tx(&k_full[st], bytes);
-                for (int k = 0; k < npg; ++k) {
-                    if (pages[k] < 0)
-                        continue;
-                    const int32_t row = (pages[k] * a.H + h) * P;
-                    for (int hf = 0; hf < 2; ++hf)
-                        tma_load_2d(&tm_kp, kdst + hf * kHalf + k * P * 128, &k_full[st], hf * 64, row);
-                }
-                mbar_arrive_expect_tx(&v_full[st], bytes);
-                for (int k = 0; k < npg; ++k) {
-                    if (pages[k] < 0)
-                        continue;
-                    const int32_t row = (pages[k] * a.H + h) * P;
-                    for (int hf = 0; hf < 2; ++hf)
-                        tma_load_2d(&tm_vp, vdst + hf * kHalf + k * P * 128, &v_full[st], hf * 64, row);
-                }
+                mbar_arrive_expect_tx(&full[st], bytes);
+                for (int k = 0; k < npg; ++k)
+                    if (pages[k] >= 0)
+                        for (int hf = 0; hf < 2; ++hf)
+                            tma_load_2d(tm_pages, dst + hf * kHalf + k * P * 128, &full[st], hf * 64,
+                                        (pages[k] * a.H + h) * P);
             } else {
                 const int32_t row = (int32_t)(g.key_row0 + (tg.j0 - g.C));
-                mbar_arrive_expect_tx(&k_full[st], 2 * kHalf);
+                mbar_arrive_expect_tx(&full[st], kTileBytes);
                 for (int hf = 0; hf < 2; ++hf)
-                    tma_load_3d(&tm_k, kdst + hf * kHalf, &k_full[st], hf * 64, h, row);
-                mbar_arrive_expect_tx(&v_full[st], 2 * kHalf);
-                for (int hf = 0; hf < 2; ++hf)
-                    tma_load_3d(&tm_v, vdst + hf * kHalf, &v_full[st], hf * 64, h, row);
+                    tma_load_3d(tm_rows, dst + hf * kHalf, &full[st], hf * 64, h, row);
             }
             issued = t + 1;
         }
         // drain: loads still in flight must land before the CTA may exit (a local flag, so
         // the drain itself never raises the CTA-wide abort)
         volatile int never = 0;
-        mbar_wait(q_full, 0, &never, tmo);
-        for (int t = (issued > kStages ? issued - kStages : 0); t < issued; ++t) {
-            const int st = t % kStages;
-            const uint32_t kph = (t / kStages) & 1;
-            mbar_wait(&k_full[st], kph, &never, tmo);
-            mbar_wait(&v_full[st], kph, &never, tmo);
-        }
+        if (!is_v)
+            mbar_wait(q_full, 0, &never, tmo);
+        for (int t = (issued > stages ? issued - stages : 0); t < issued; ++t)
+            mbar_wait(&full[t % stages], (t / stages) & 1, &never, tmo);
     } else if (warp == 1 && lane == 0) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
         const uint32_t qbase = sbase + kOffQ;
-        const uint32_t pbase = sbase + kOffP;
         bool ok = mbar_wait(q_full, 0, abort_flag, tmo);
         auto issue_pv = [&](int u) -> bool {
-            const int st = u % kStages;
-            const uint32_t kph = (u / kStages) & 1;
-            if (!mbar_wait(p_full, u & 1, abort_flag, tmo))
+            const int vst = u % kVStages;
+            const int pb = u & 1;
+            if (!mbar_wait(&p_full[pb], (u >> 1) & 1, abort_flag, tmo))
                 return false;
-            if (!mbar_wait(&v_full[st], kph, abort_flag, tmo))
+            if (!mbar_wait(&v_full[vst], (u / kVStages) & 1, abort_flag, tmo))
                 return false;
             tc_fence_after();
-            const uint32_t vbase = sbase + kOffStage + st * kStageBytes + 2 * kHalf;
+            const uint32_t vbase = sbase + kOffV + vst * kTileBytes;
+            const uint32_t pcol = tmem + (pb ? kColP1 : kColP0);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = smem_desc_sw128(pbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
                 const uint64_t bd = smem_desc_sw128(vbase + kk * 2048, kHalf, 1024);
-                umma_bf16_ss(tmem + kColO, ad, bd, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+                umma_bf16_ts(tmem + kColO, pcol + kk * 8, bd, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
             }
-            umma_commit(p_empty);
-            umma_commit(&kv_empty[st]);
+            umma_commit(&p_empty[pb]);
+            umma_commit(&v_empty[vst]);
             return true;
         };
         for (int t = 0; ok && t < n; ++t) {
-            const int st = t % kStages;
-            const uint32_t kph = (t / kStages) & 1;
+            const int kst = t % kKStages;
             const int sb = t & 1;
-            const uint32_t sph = (t >> 1) & 1;
-            if (!mbar_wait(&k_full[st], kph, abort_flag, tmo)) {
+            if (!mbar_wait(&k_full[kst], (t / kKStages) & 1, abort_flag, tmo)) {
                 ok = false;
                 break;
             }
-            if (t >= 2 && !mbar_wait(&s_empty[sb], sph ^ 1, abort_flag, tmo)) {
+            if (t >= 2 && !mbar_wait(&s_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t kbase = sbase + kOffStage + st * kStageBytes;
+            const uint32_t kbase = sbase + kOffK + kst * kTileBytes;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint64_t ad = smem_desc_sw128(qbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
@@ -377,6 +427,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 umma_bf16_ss(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
             }
             umma_commit(&s_full[sb]);
+            umma_commit(&k_empty[kst]);
             if (t >= 1 && !issue_pv(t - 1)) {
                 ok = false;
                 break;
@@ -389,11 +440,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         umma_commit(o_full);
         volatile int never = 0;
         mbar_wait(o_full, 0, &never, tmo);
-    } else if (warp == 2 || warp == 3) {
-        // ============================================================ bias window producers
-        const int ht = threadIdx.x - 64;                  // 0..63
-        named_barrier_sync(2, 320);                       // bounds and rab staged by warps 4-11
+    } else if (warp == 2) {
+        // ============================================================ bias window producer
+        const int ht = lane;                              // 0..31
         const int nb = a.NB;
+        const float lg_scale = a.ln_nmax > 0.0 ? (float)((double)(nb - 1) * 0.6931471805599453 / a.ln_nmax) : 0.f;
         bool ok = true;
         for (int t = 0; t < n; ++t) {
             const int wb = t & 1;
@@ -405,10 +456,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
             const int32_t dist0 = i0 - tg.j0 + (kTile - 1);       // distance at window index 0
             float* wbuf = win + wb * (kWinBuf / 4);
-            for (int y = ht; y < 256; y += 64) {
+#pragma unroll
+            for (int yy = 0; yy < 8; ++yy) {
+                const int y = ht + 32 * yy;
                 const int32_t d = dist0 - y;
-                const float val = (y <= 2 * kTile - 2 && d >= 0) ? 0.5f * s_rab[bucket_from_bounds(s_bounds, nb, d)]
-                                                                 : 0.f;
+                const float val = (y <= 2 * kTile - 2 && d >= 0) ? s_rab[bucket_fast(s_bounds, nb, d, lg_scale)] : 0.f;
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
                     if (y - s >= 0)
@@ -419,13 +471,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp >= 4) {
         // ============================================================ pointwise + epilogue
         const int pt = threadIdx.x - 128;                 // 0..255
-        // stage rab[h][:] and the bucket bounds, then release the bias producers
-        for (int k = pt; k < a.NB; k += 256)
-            s_rab[k] = a.rab[(int64_t)h * a.NB + k];
-        for (int k = pt; k <= a.NB; k += 256)
-            s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB, a.n_max));
-        named_barrier_sync(2, 320);
-
         const int wg = (warp - 4) >> 2;                   // key-column half
         const int r = ((warp & 3) << 5) + lane;           // query row in the block (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -437,12 +482,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int y0 = (kTile - 1) - r + 64 * wg;
         const int wsel = y0 & 3;
         const int woff = wsel * kWinStride + (y0 - wsel);
-        uint8_t* pbuf = smem + kOffP + wg * kHalf + r * 128;
-        const uint64_t half2 = f2pack(0.5f, 0.5f);
         bool ok = true;
         for (int t = 0; t < n; ++t) {
-            const int st = t % kStages;
-            const uint32_t kph = (t / kStages) & 1;
+            const int vst = t % kVStages;
             const int sb = t & 1;
             const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
             ok = ok && mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
@@ -451,76 +493,60 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!ok)
                 break;
             tc_fence_after();
-            uint32_t sv[64];
-            const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0) + wg * 64;
-            tmem_ld_32x32b_x32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld_32x32b_x32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&s_empty[sb]);
-
             const float4* wv = reinterpret_cast<const float4*>(win + sb * (kWinBuf / 4) + woff);
             const bool full = (qrow0 + kTile - 1 < g.N) && (tg.j0 + kTile - 1 < tg.kvend) &&
                               (tg.j0 + kTile - 1 <= i0) && (tg.j0 + kTile - 1 < g.hist);
             const int32_t lim = min(lim_row, tg.kvend);
             const int32_t diag = (row_valid && !tg.cached) ? i_abs : -1;
             const int jc0 = tg.j0 + wg * 64;                  // key position of column 0 of this half
+            const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0) + wg * 64;
+            uint32_t sv[32], sv2[32];
             uint32_t packed[32];
-#pragma unroll
-            for (int q4 = 0; q4 < 16; ++q4) {
-                const float4 bias = wv[q4];
-                // x/2 = S/2 + rab/2 for four columns, as two packed pairs
-                const uint64_t xa = f2fma(f2pack(__uint_as_float(sv[4 * q4]), __uint_as_float(sv[4 * q4 + 1])), half2,
-                                          f2pack(bias.x, bias.y));
-                const uint64_t xb = f2fma(f2pack(__uint_as_float(sv[4 * q4 + 2]), __uint_as_float(sv[4 * q4 + 3])),
-                                          half2, f2pack(bias.z, bias.w));
-                float a0, a1, a2, a3;
-                f2unpack(xa, a0, a1);
-                f2unpack(xb, a2, a3);
-                // SiLU(x) = x/2 * (1 + tanh(x/2))
-                const uint64_t wa = f2fma(xa, f2pack(tanh_approx(a0), tanh_approx(a1)), xa);
-                const uint64_t wb2 = f2fma(xb, f2pack(tanh_approx(a2), tanh_approx(a3)), xb);
-                float w0, w1, w2, w3;
-                f2unpack(wa, w0, w1);
-                f2unpack(wb2, w2, w3);
-                if (!full) {
-                    const int j = jc0 + 4 * q4;
-                    w0 = ((j < lim) || (j == diag)) ? w0 : 0.f;
-                    w1 = ((j + 1 < lim) || (j + 1 == diag)) ? w1 : 0.f;
-                    w2 = ((j + 2 < lim) || (j + 2 == diag)) ? w2 : 0.f;
-                    w3 = ((j + 3 < lim) || (j + 3 == diag)) ? w3 : 0.f;
-                }
-                packed[2 * q4] = bf16x2_rn(w0, w1);
-                packed[2 * q4 + 1] = bf16x2_rn(w2, w3);
-            }
+            // first 32 columns: load, wait; then start the second load and compute the first half
+            tmem_ld_32x32b_x32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_wait_ld();
+            tmem_ld_32x32b_x32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv2[0]));
+            if (full)
+                silu_cols32<false>(sv, wv, packed, jc0, lim, diag);
+            else
+                silu_cols32<true>(sv, wv, packed, jc0, lim, diag);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&s_empty[sb]);
+            if (full)
+                silu_cols32<false>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag);
+            else
+                silu_cols32<true>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag);
             mbar_arrive(&win_empty[sb]);
-            if (t >= 1) {
-                ok = ok && mbar_wait(p_empty, (t - 1) & 1, abort_flag, tmo);
+            // P buffer sb is free once P V of tile t - 2 completed
+            if (t >= 2) {
+                ok = ok && mbar_wait(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
             }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                uint4 v4 = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-                *reinterpret_cast<uint4*>(pbuf + ((q ^ (r & 7)) << 4)) = v4;
-            }
+            tmem_st_32x32b_x32(tmem + lane_base + (sb ? kColP1 : kColP0) + wg * 32,
+                               *reinterpret_cast<const uint32_t(*)[32]>(&packed[0]));
             const int vz = tg.kvend - tg.j0;                   // valid key rows in this tile
             if (vz < kTile) {
-                ok = ok && mbar_wait(&v_full[st], kph, abort_flag, tmo);
+                // rows past the valid keys may hold anything (page tails, other users): zero
+                // them so that 0 * NaN cannot reach O
+                ok = ok && mbar_wait(&v_full[vst], (t / kVStages) & 1, abort_flag, tmo);
                 if (ok) {
-                    uint8_t* vt = smem + kOffStage + st * kStageBytes + 2 * kHalf;
+                    uint8_t* vt = smem + kOffV + vst * kTileBytes;
                     const int first = vz > 0 ? vz : 0;
                     const int nchunks = (kTile - first) * 16;
                     for (int x = pt; x < nchunks; x += 256) {
                         const int row = first + (x >> 4), hf = (x >> 3) & 1, ch = x & 7;
                         *reinterpret_cast<uint4*>(vt + hf * kHalf + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
                     }
+                    fence_proxy_async_smem();
                 }
             }
+            tmem_wait_st();
             if (ok) {
-                fence_proxy_async_smem();
-                mbar_arrive(p_full);
+                tc_fence_before();
+                mbar_arrive(&p_full[sb]);
             }
         }
         // ------------------------------------------------------------ epilogue: O / n_max -> workspace
@@ -558,7 +584,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host side
-void launch_attn_tc(const TcMaps& m, const TcArgs& a, bool paged, int32_t B, cudaStream_t stream)
+
+void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
+                    cudaStream_t stream)
 {
     static bool attr_set[2] = {false, false};
     const int64_t grid_x = (int64_t)a.splits * a.H * B;
@@ -570,13 +598,13 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, bool paged, int32_t B, cud
             cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             attr_set[1] = true;
         }
-        attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, a);
+        attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
     } else {
         if (!attr_set[0]) {
             cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             attr_set[0] = true;
         }
-        attn_tc_kernel<false><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, a);
+        attn_tc_kernel<false><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
     }
 }
 

@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/hstu.h"
+#include "hstu.h"
 
 namespace hstu {
 

@@ -42,6 +42,15 @@ struct TcMaps {
     CUtensorMap q, k, v, kp, vp;
 };
 
+// Bucket boundaries computed on the host: v[k] = smallest distance d with bucket(d) >= k for
+// k < count - 1, v[count - 1] = INT_MAX.  count == 0 means "not passed" (too many buckets for
+// the parameter block); the kernels then evaluate them on the device.
+constexpr int kMaxParamNB = 512;
+struct BucketBounds {
+    int32_t count;
+    int32_t v[kMaxParamNB + 1];
+};
+
 void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, const void* k_new,
                       const void* v_new, const int32_t* cached_lens, const int32_t* new_lens,
                       const int32_t* num_targets, int32_t B, int64_t total_new, int32_t H, int32_t D,
@@ -51,6 +60,7 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
 void launch_ln_gate(const float* part, int32_t S, int64_t ntok, int32_t HD, const void* u, void* out, bool fp32,
                     float eps, cudaStream_t stream);
 void launch_attn_simt(const SimtArgs& a, bool paged, bool fp32, int32_t B, cudaStream_t stream);
-void launch_attn_tc(const TcMaps& m, const TcArgs& a, bool paged, int32_t B, cudaStream_t stream);
+void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
+                    cudaStream_t stream);
 
 }  // namespace hstu
