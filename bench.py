@@ -173,15 +173,32 @@ def setup_device(layers, device):
     return p, ws, kp, vp, L
 
 
-def run_step(hb, p, ws, kp, vp, L, max_new, events=None):
+def run_step(hb, p, ws, kp, vp, L, max_new, events=None, side=None):
+    """One step: per layer kv_append of the 16 new history tokens and paged attention of all
+    80 new tokens.  The attention reads the new keys from k_new/v_new, not from the pages, so
+    the appends do not feed it: with a side stream they run concurrently (fork at the start of
+    the step, join at the end)."""
+    import torch
+
+    main = torch.cuda.current_stream()
+    if side is not None:
+        side.wait_stream(main)
     for li, t in enumerate(L):
-        hb.kv_append(p, kp, vp, t["pt"], t["k"], t["v"], t["cl"], t["nl"], t["nt"], max_new=max_new, workspace=ws)
+        if side is not None:
+            with torch.cuda.stream(side):
+                hb.kv_append(p, kp, vp, t["pt"], t["k"], t["v"], t["cl"], t["nl"], t["nt"], max_new=max_new,
+                             workspace=ws, stream=side)
+        else:
+            hb.kv_append(p, kp, vp, t["pt"], t["k"], t["v"], t["cl"], t["nl"], t["nt"], max_new=max_new,
+                         workspace=ws)
         if events is not None:
             events[li][0].record()
         hb.paged_fwd(p, t["q"], t["k"], t["v"], t["u"], kp, vp, t["pt"], t["cl"], t["nl"], t["nt"], t["rab"],
                      max_new=max_new, workspace=ws, out=t["out"])
         if events is not None:
             events[li][1].record()
+    if side is not None:
+        main.wait_stream(side)
 
 
 def bench_prefill(hb, device, steps, warmup, peaks):
@@ -246,6 +263,39 @@ def cpu_oracle_layer(layer, nthreads=None):
     return time.perf_counter() - t0
 
 
+def profile_case(case, calls):
+    """A small case for ncu: `calls` launches of one layer of the paged batch (its own pages
+    only, ~0.4 GB on the device) or of the jagged prefill batch."""
+    import torch
+
+    import hstu_attention_b200 as hb
+
+    torch.cuda.set_device(0)
+    if case == "paged":
+        c = gen.config3_paged_layers(layers=1)[0]
+        ck, cv, cpt = c.compact_pool()
+        import dataclasses
+
+        compact = dataclasses.replace(c, num_pages=int(ck.shape[0]), page_table=cpt,
+                                      page_ids=np.arange(ck.shape[0], dtype=np.int32))
+        p, ws, kp, vp, L = setup_device([compact], torch.device("cuda", 0))
+        t = L[0]
+        for _ in range(calls):
+            hb.paged_fwd(p, t["q"], t["k"], t["v"], t["u"], kp, vp, t["pt"], t["cl"], t["nl"], t["nt"], t["rab"],
+                         max_new=c.max_new, workspace=ws, out=t["out"])
+    else:
+        c = gen.config2_prefill()
+        d = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)  # noqa
+        p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max)
+        ws = hb.Workspace(p, c.B, c.T, 4096)
+        args = (d(c.q), d(c.k), d(c.v), d(c.u), torch.from_numpy(c.seq_offsets.astype(np.int32)).cuda(),
+                torch.from_numpy(c.num_targets.astype(np.int32)).cuda(), torch.from_numpy(c.rab).cuda())
+        for _ in range(calls):
+            hb.jagged_fwd(p, *args, max_seqlen=4096, workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -255,7 +305,13 @@ def main():
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["paged", "prefill"], default=None,
+                    help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
+    ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case, args.calls)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -318,9 +374,10 @@ def main():
     # each paged attention call (external events: recorded as graph nodes)
     events = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
               for _ in L]
+    side = torch.cuda.Stream(device=device)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        run_step(hb, p, ws, kp, vp, L, max_new, events=events)
+        run_step(hb, p, ws, kp, vp, L, max_new, events=events, side=side)
     graph.replay()
     torch.cuda.synchronize()
 
@@ -429,7 +486,8 @@ def main():
                    "global_batch": layers_cfg["B"] * world, "seq_len": int(max(int(c.cached_lens.max()) for c in layers)),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (8 layers of distinct pages, ~370 MB per step)",
-                   "graph": "one CUDA graph per step"},
+                   "graph": "one CUDA graph per step; appends on a forked stream (they do not feed "
+                            "the attention, which reads new keys from k_new)"},
         "roofline": {"bound": "hbm", "kernel": "hstu_attn_paged_fwd (attention kernel + LayerNorm-gate kernel)",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
                      "peak_kind": peaks_kind, "algorithmic_bytes_per_call": mean_bytes,

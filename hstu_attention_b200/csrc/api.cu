@@ -141,20 +141,6 @@ static int num_sms()
     return cached;
 }
 
-// Split of each (user, head, query block)'s keys over CTAs for the paged tensor-core path:
-// enough CTAs to cover the SMs once, at most kMaxSplits.
-static int paged_splits(const hstu_attn_params* p, int32_t B, int32_t max_new)
-{
-    const int64_t qblocks = (max_new + 127) / 128;
-    const int64_t units = (int64_t)B * p->num_heads * (qblocks > 0 ? qblocks : 1);
-    int64_t s = units > 0 ? num_sms() / units : 1;
-    if (s < 1)
-        s = 1;
-    if (s > kMaxSplits)
-        s = kMaxSplits;
-    return (int)s;
-}
-
 static size_t partial_bytes(const hstu_attn_params* p, int splits, int64_t tokens)
 {
     return (size_t)splits * (size_t)tokens * (size_t)p->num_heads * (size_t)p->head_dim * sizeof(float);
@@ -239,10 +225,10 @@ size_t hstu_workspace_size(const hstu_attn_params* params, int32_t max_batch, in
 {
     if (check_params(params, false) != HSTU_OK || max_batch < 0 || max_tokens < 0 || max_new < 0)
         return 0;
-    int splits = 1;
-    if (use_tc(params))
-        splits = paged_splits(params, max_batch > 0 ? max_batch : 1, max_new);
-    size_t bytes = kStatusBytes + partial_bytes(params, splits, max_tokens);
+    // the tensor-core paged path spreads a user's keys over up to kMaxSplits CTAs, each with
+    // its own fp32 partial plane; every other path writes one plane
+    const int planes = use_tc(params) ? kMaxSplits : 1;
+    size_t bytes = kStatusBytes + counts_bytes(max_tokens) + partial_bytes(params, planes, max_tokens);
     return (bytes + 255) & ~(size_t)255;
 }
 
@@ -326,8 +312,9 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         return HSTU_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out))
         return HSTU_ERR_INVALID_ARG;
-    if (workspace_bytes < kStatusBytes + partial_bytes(params, 1, total_tokens))
+    if (workspace_bytes < kStatusBytes + counts_bytes(total_tokens) + partial_bytes(params, 1, total_tokens))
         return HSTU_ERR_WORKSPACE;
+    float* part = partials(workspace, total_tokens);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const double ln_nmax = log((double)params->n_max);
     const bool fp32 = params->dtype == HSTU_DTYPE_FP32;
@@ -344,6 +331,8 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.num_targets = num_targets;
         a.rab = rab;
         a.ws = workspace;
+        a.part = part;
+        a.counts = nullptr;
         a.total_tokens = total_tokens;
         a.max_len = max_seqlen;
         a.H = params->num_heads;
@@ -352,7 +341,9 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.P = 1;
         a.num_pages = 0;
         a.max_pages = 0;
-        a.splits = 1;
+        a.B = B;
+        a.max_splits = 1;
+        a.target_ctas = num_sms();
         a.qblocks = (max_seqlen + 127) / 128;
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
@@ -367,6 +358,7 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.num_targets = num_targets;
         a.rab = rab;
         a.ws = workspace;
+        a.part = part;
         a.total_tokens = total_tokens;
         a.max_len = max_seqlen;
         a.H = params->num_heads;
@@ -377,8 +369,8 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.ln_nmax = ln_nmax;
         launch_attn_simt(a, false, fp32, B, s);
     }
-    launch_ln_gate(partials(workspace), 1, total_tokens, params->num_heads * params->head_dim, u, out, fp32,
-                   params->ln_eps, s);
+    launch_ln_gate(part, 1, nullptr, total_tokens, params->num_heads * params->head_dim, u, out, fp32, params->ln_eps,
+                   s);
     return finish(s);
 }
 
@@ -404,17 +396,20 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         !aligned16(v_pages) || !aligned16(out))
         return HSTU_ERR_INVALID_ARG;
     const size_t one = partial_bytes(params, 1, total_new);
-    if (workspace_bytes < kStatusBytes + one)
+    const size_t fixed = kStatusBytes + counts_bytes(total_new);
+    if (workspace_bytes < fixed + one)
         return HSTU_ERR_WORKSPACE;
+    float* part = partials(workspace, total_new);
+    int32_t* counts = split_counts(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const double ln_nmax = log((double)params->n_max);
     const bool fp32 = params->dtype == HSTU_DTYPE_FP32;
     int splits = 1;
     if (use_tc(params)) {
-        splits = paged_splits(params, B, max_new);
-        const int fit = (int)((workspace_bytes - kStatusBytes) / one);
-        if (splits > fit)
-            splits = fit;
+        // as many partial planes as the workspace holds, up to kMaxSplits
+        splits = (int)((workspace_bytes - fixed) / one);
+        if (splits > kMaxSplits)
+            splits = kMaxSplits;
         TcMaps m;
         const int64_t page_rows = (int64_t)params->num_pages * params->num_heads * params->page_size;
         if (!encode_rows(&m.q, q_new, total_new, params->num_heads, 128) ||
@@ -430,6 +425,8 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.page_table = page_table;
         a.rab = rab;
         a.ws = workspace;
+        a.part = part;
+        a.counts = counts;
         a.total_tokens = total_new;
         a.max_len = max_new;
         a.H = params->num_heads;
@@ -438,7 +435,9 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.P = params->page_size;
         a.num_pages = params->num_pages;
         a.max_pages = params->max_pages_per_user;
-        a.splits = splits;
+        a.B = B;
+        a.max_splits = splits;
+        a.target_ctas = num_sms();
         a.qblocks = (max_new + 127) / 128;
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
@@ -457,6 +456,7 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.num_targets = num_targets;
         a.rab = rab;
         a.ws = workspace;
+        a.part = part;
         a.total_tokens = total_new;
         a.max_len = max_new;
         a.H = params->num_heads;
@@ -469,8 +469,8 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.ln_nmax = ln_nmax;
         launch_attn_simt(a, true, fp32, B, s);
     }
-    launch_ln_gate(partials(workspace), splits, total_new, params->num_heads * params->head_dim, u_new, out, fp32,
-                   params->ln_eps, s);
+    launch_ln_gate(part, splits, use_tc(params) ? counts : nullptr, total_new, params->num_heads * params->head_dim,
+                   u_new, out, fp32, params->ln_eps, s);
     return finish(s);
 }
 

@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtArgs a)
         return;                                // past this user's queries (uniform)
     const bool row_ok = tq < g.N;
     const int i = g.C + tq;                    // absolute position
-    float* out = partials(a.ws);
+    float* out = a.part;
 
     float acc[kSimtMaxD / 4];
 #pragma unroll

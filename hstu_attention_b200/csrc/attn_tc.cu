@@ -55,7 +55,8 @@ constexpr uint32_t kTileBytes = 2 * kHalf;    // one 128 x 128 bf16 operand
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTileBytes;
 constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
-constexpr uint32_t kWinStride = 260;          // floats per shifted copy (256 + 4: spreads banks)
+constexpr uint32_t kWinPad = 4;               // floats before each shifted copy (stores at y - s >= -3)
+constexpr uint32_t kWinStride = 264;          // floats per copy: pad + 256 + 4 (spreads banks)
 constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
 constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
@@ -93,26 +94,29 @@ __device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t ct, int32_t C, in
     return g;
 }
 
-// bucket(d) from a float estimate of the log-spaced index, corrected against the exact
-// bounds (bounds[k] = smallest d with bucket(d) >= k, bounds[nb] a sentinel).  The estimate's
-// error is far below one bucket, so one step of correction suffices.
-// lg_scale = (nb - 1) / log2(n_max).
-__device__ __forceinline__ int bucket_fast(const int32_t* bounds, int nb, int32_t d, float lg_scale)
+// bucket(d) for eight distances at once: the largest k with bounds[k] <= d, where bounds[k]
+// is the smallest distance in bucket k (bounds[0] = 0, bounds[nb] = INT_MAX, d < 0 -> 0).
+// A branchless binary search on shared memory, the eight searches interleaved so their load
+// latencies overlap.  Only integer and load instructions: the special-function pipe stays
+// free for the pointwise warps' tanh.
+__device__ __forceinline__ void bucket_search8(const int32_t* bounds, int nb, int top, const int32_t (&d)[8],
+                                               int (&k)[8])
 {
-    if (d <= 0 || nb <= 1)
-        return 0;
-    int b = 1 + __float2int_rd(__log2f((float)d) * lg_scale);
-    b = max(1, min(b, nb - 1));
-    if (d < bounds[b])
-        --b;
-    else if (d >= bounds[b + 1])
-        ++b;
-    return b;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        k[e] = 0;
+    // Written without short-circuit logic: a data-dependent && / || here compiles to branches
+    // that diverge across lanes and serialise the warp.
+    for (int step = top; step > 0; step >>= 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            k[e] += (bounds[min(k[e] + step, nb)] <= d[e]) ? step : 0;
+    }
 }
 
 // SiLU weights of 32 consecutive key columns of one query row: x/2 = S/2 + bias (bias holds
 // rab/2), w = x/2 * (1 + tanh(x/2)), masked to 0 where the key is not visible, packed to
-// bf16x2.
+// bf16x2 with integer rounding (see bf16x2_round_int).
 // kMasked selects the per-column visibility test at compile time, so the full-tile loop has
 // no branch and the compiler can interleave the independent tanh chains.
 template <bool kMasked>
@@ -136,14 +140,14 @@ __device__ __forceinline__ void silu_cols32(const uint32_t* sv, const float4* wv
         f2unpack(wa, w0, w1);
         f2unpack(wb, w2, w3);
         if (kMasked) {
-            const int j = jc + 4 * q4;
-            w0 = ((j < lim) || (j == diag)) ? w0 : 0.f;
-            w1 = ((j + 1 < lim) || (j + 1 == diag)) ? w1 : 0.f;
-            w2 = ((j + 2 < lim) || (j + 2 == diag)) ? w2 : 0.f;
-            w3 = ((j + 3 < lim) || (j + 3 == diag)) ? w3 : 0.f;
+            const int j = jc + 4 * q4;           // bitwise | : no lane-divergent branches
+            w0 = ((j < lim) | (j == diag)) ? w0 : 0.f;
+            w1 = ((j + 1 < lim) | (j + 1 == diag)) ? w1 : 0.f;
+            w2 = ((j + 2 < lim) | (j + 2 == diag)) ? w2 : 0.f;
+            w3 = ((j + 3 < lim) | (j + 3 == diag)) ? w3 : 0.f;
         }
-        packed[2 * q4] = bf16x2_rn(w0, w1);
-        packed[2 * q4 + 1] = bf16x2_rn(w2, w3);
+        packed[2 * q4] = bf16x2_round_int(w0, w1);
+        packed[2 * q4 + 1] = bf16x2_round_int(w2, w3);
     }
 }
 
@@ -166,6 +170,118 @@ __device__ int bucket_bound(int k, double ln_nmax, int nb)
     return c > 0x7ffffffe ? 0x7ffffffe : (int)c;
 }
 
+// ------------------------------------------------------------------ paged work plan
+// Entry e = user * qblocks + q-block.  Key tiles of an entry: the cached tiles plus the new-key
+// tiles up to the block's last query (qblk + 1 of them).  A user with invalid lengths keeps
+// one tile on q-block 0 so that one CTA writes its (zero) rows and flags it.
+__device__ __forceinline__ int entry_tiles(const TcArgs& a, int e)
+{
+    const int b = e / a.qblocks, q = e % a.qblocks;
+    const int32_t C = a.cached_lens[b], N = a.new_lens[b];
+    const int32_t T = a.num_targets ? a.num_targets[b] : 0;
+    const bool ok = C >= 0 && N >= 0 && T >= 0 && T <= N && N <= a.max_len && C <= a.max_pages * a.P;
+    if (!ok)
+        return q == 0 ? 1 : 0;
+    if (q * kTile >= N)
+        return 0;
+    return (C + kTile - 1) / kTile + q + 1;
+}
+
+// The entries' tile counts of this lane (entries lane, lane + 32, ...), read once.  Entries
+// past kPlanRounds * 32 are re-read when needed (the arrays are then in L1).
+constexpr int kPlanRounds = 8;
+struct PlanTiles {
+    int t[kPlanRounds];
+};
+
+__device__ __forceinline__ int splits_for(int t, int c, int max_splits)
+{
+    return t == 0 ? 0 : min((t + c - 1) / c, max_splits);
+}
+
+// Tiles per piece c: start from ceil(all tiles over all heads / target_ctas) and grow until
+// the pieces fit the grid that was launched (gridDim.x >= H * entries bounds the count at
+// c = max tiles, so a fit always exists).  Whole warp.
+__device__ int plan_tiles_per_piece(const TcArgs& a, const PlanTiles& pt)
+{
+    const int lane = threadIdx.x & 31;
+    const int entries = a.B * a.qblocks;
+    int64_t w = 0;
+#pragma unroll
+    for (int r = 0; r < kPlanRounds; ++r)
+        w += pt.t[r];                                    // zero past the last entry
+    for (int e = lane + 32 * kPlanRounds; e < entries; e += 32)
+        w += entry_tiles(a, e);
+    for (int o = 16; o > 0; o >>= 1)
+        w += __shfl_xor_sync(0xffffffffu, w, o);
+    w *= a.H;
+    const int64_t tgt = a.target_ctas > 0 ? a.target_ctas : 1;
+    int c = (int)((w + tgt - 1) / tgt);
+    if (c < 1)
+        c = 1;
+    for (int it = 0; it < 64; ++it) {
+        int64_t units = 0;
+#pragma unroll
+        for (int r = 0; r < kPlanRounds; ++r)
+            units += splits_for(pt.t[r], c, a.max_splits);
+        for (int e = lane + 32 * kPlanRounds; e < entries; e += 32)
+            units += splits_for(entry_tiles(a, e), c, a.max_splits);
+        for (int o = 16; o > 0; o >>= 1)
+            units += __shfl_xor_sync(0xffffffffu, units, o);
+        if (units * a.H <= (int64_t)gridDim.x)
+            return c;
+        c += (c + 7) / 8;                     // grow by ~12% per step
+    }
+    return 0x3fffffff;                        // one piece per entry always fits the grid
+}
+
+// The piece this CTA (blockIdx.x) works on: entry e_out, index local_out within the entry and
+// the entry's number of splits (pieces are numbered entry by entry, H * splits(e) per entry).
+// Returns false past the last piece.  Whole warp.
+__device__ bool plan_unit(const TcArgs& a, int& e_out, int& local_out, int& nsplit_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int entries = a.B * a.qblocks;
+    PlanTiles pt;
+#pragma unroll
+    for (int r = 0; r < kPlanRounds; ++r) {
+        const int e = lane + 32 * r;
+        pt.t[r] = e < entries ? entry_tiles(a, e) : 0;
+    }
+    const int c = plan_tiles_per_piece(a, pt);
+    const int want = (int)blockIdx.x;
+    int base = 0;
+    for (int r0 = 0, r = 0; r0 < entries; r0 += 32, ++r) {
+        const int e = r0 + lane;
+        int t = 0;
+#pragma unroll
+        for (int k = 0; k < kPlanRounds; ++k)
+            t = (k == r) ? pt.t[k] : t;                  // register select, no local memory
+        if (r >= kPlanRounds && e < entries)
+            t = entry_tiles(a, e);
+        const int ns = e < entries ? splits_for(t, c, a.max_splits) : 0;
+        const int units = a.H * ns;
+        int incl = units;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += y;
+        }
+        const int excl = incl - units;
+        const bool mine = units > 0 && want >= base + excl && want < base + incl;
+        const unsigned who = __ballot_sync(0xffffffffu, mine);
+        if (who) {
+            const int src = __ffs(who) - 1;
+            e_out = __shfl_sync(0xffffffffu, e, src);
+            local_out = __shfl_sync(0xffffffffu, want - base - excl, src);
+            nsplit_out = __shfl_sync(0xffffffffu, ns, src);
+            return true;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return false;
+}
+
 template <bool kPaged>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -177,12 +293,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ UserGeom sG;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // grid: x = (split, head, user) fastest-varying, y = query block, heaviest blocks first
-    const int split = blockIdx.x % a.splits;
-    const int h = (blockIdx.x / a.splits) % a.H;
-    const int b = blockIdx.x / (a.splits * a.H);
-    const int qblk = a.qblocks - 1 - (int)blockIdx.y;
+    __shared__ int sUnit[5];
+    int b, qblk, h, split, nsplit;
+    if (kPaged) {
+        // balanced work plan: every (user, query block) entry's key tiles are cut into
+        // ceil(tiles / c) contiguous pieces, c chosen so that about target_ctas pieces exist
+        // over all heads; this CTA takes piece blockIdx.x (computed the same way by every CTA)
+        if (warp == 0) {
+            int e = -1, local = 0, ns = 1;
+            const bool found = plan_unit(a, e, local, ns);
+            if (lane == 0) {
+                sUnit[0] = found ? e : -1;                     // entry: user * qblocks + q-block
+                sUnit[1] = local;                              // piece index within the entry
+                sUnit[2] = found ? ns : 1;
+            }
+        }
+        __syncthreads();
+        if (sUnit[0] < 0) {
+            pdl_launch_dependents();
+            return;                                  // more CTAs than pieces
+        }
+        const int e = sUnit[0], local = sUnit[1];
+        b = e / a.qblocks;
+        qblk = e % a.qblocks;
+        nsplit = sUnit[2];
+        h = local / nsplit;
+        split = local % nsplit;
+    } else {
+        // grid: x = (head, user), y = query block, heaviest blocks first
+        h = blockIdx.x % a.H;
+        b = blockIdx.x / a.H;
+        qblk = a.qblocks - 1 - (int)blockIdx.y;
+        split = 0;
+        nsplit = 1;
+    }
 
+    extern __shared__ __align__(1024) uint8_t smem_pre[];
+    if (kPaged && (warp == 2 || warp == 3)) {
+        // the user's page-table row, loaded while warp 0 reads the lengths (page ids past the
+        // user's cached length are never used; invalid ids are caught when a page is used)
+        const uint32_t pre_pad = (1024u - (sm100::smem_u32(smem_pre) & 1023u)) & 1023u;
+        int32_t* rowbuf = reinterpret_cast<int32_t*>(smem_pre + pre_pad + kOffPages);
+        const int nrow = min(a.max_pages, kMaxPageIds);
+        for (int k = threadIdx.x - 64; k < nrow; k += 64)
+            rowbuf[k] = a.page_table[(int64_t)b * a.max_pages + k];
+    }
     if (warp == 0) {
         const bool report = qblk == 0 && h == 0 && split == 0;
         UserGeom g = kPaged ? paged_geom(a.cached_lens, a.new_lens, a.num_targets, b, a.total_tokens, a.max_len,
@@ -195,8 +350,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     const UserGeom g = sG;
     const int32_t qrow0 = qblk * kTile;
-    if (qrow0 >= g.N)
+    if (qrow0 >= g.N) {
+        pdl_launch_dependents();
         return;                                               // no queries here (uniform)
+    }
 
     const int32_t i0 = g.C + qrow0;                           // absolute position of row 0
     const int32_t last_q = min(g.N, qrow0 + kTile) - 1;
@@ -204,11 +361,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int32_t ct = kPaged ? (g.C + kTile - 1) / kTile : 0;
     const int32_t nnew = kend > g.C ? (kend - g.C + kTile - 1) / kTile : 0;
     const int32_t ntot = ct + nnew;
-    const int32_t t_begin = (int32_t)(((int64_t)ntot * split) / a.splits);
-    const int32_t t_end = (int32_t)(((int64_t)ntot * (split + 1)) / a.splits);
+    const int32_t t_begin = (int32_t)(((int64_t)ntot * split) / nsplit);
+    const int32_t t_end = (int32_t)(((int64_t)ntot * (split + 1)) / nsplit);
     const int32_t n = g.ok ? t_end - t_begin : 0;
     const int64_t HD = (int64_t)a.H * kTcD;
-    float* part = partials(a.ws) + (int64_t)split * a.total_tokens * HD;
+    float* part = a.part + (int64_t)split * a.total_tokens * HD;
+    if (kPaged && h == 0 && split == 0) {
+        // the LayerNorm kernel sums this many partial planes for each of these tokens
+        for (int r = threadIdx.x; r < kTile; r += kTcThreads)
+            if (qrow0 + r < g.N)
+                a.counts[g.tok0 + qrow0 + r] = g.ok ? nsplit : 1;
+    }
 
     if (n <= 0) {
         // nothing to accumulate: this split's partial rows are zero
@@ -218,6 +381,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + r) * HD + (int64_t)h * kTcD)[c4] =
                     make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        pdl_launch_dependents();
         return;
     }
 
@@ -280,27 +444,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == 2 || warp == 3) {
         const int ht = threadIdx.x - 64;
         if (kPaged) {
-            // this CTA's page ids (validated; -1 = skip the load)
-            for (int k = ht; k < lp_end - lp_begin && k < kMaxPageIds; k += 64) {
-                int32_t pg = a.page_table[(int64_t)b * a.max_pages + lp_begin + k];
+            // validate the staged page ids this CTA will use (-1 = skip the load)
+            for (int k = lp_begin + ht; k < lp_end && k < kMaxPageIds; k += 64) {
+                const int32_t pg = s_pages[k];
                 if (pg < 0 || pg >= a.num_pages) {
                     set_flag(a.ws, HSTU_DEV_BAD_PAGE);
-                    pg = -1;
+                    s_pages[k] = -1;
                 }
-                s_pages[k] = pg;
             }
         }
-        for (int k = ht; k < a.NB; k += 64)
-            s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
-        if (bb.count > 0) {
-            for (int k = ht; k <= a.NB; k += 64)
-                s_bounds[k] = bb.v[k];
-        }
-    }
-    if (bb.count == 0 && warp >= 4) {
-        // bounds not passed by the host (many buckets): evaluate them here
-        for (int k = threadIdx.x - 128; k <= a.NB; k += 256)
-            s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB));
     }
     tc_fence_before();
     __syncthreads();
@@ -346,9 +498,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const int lp = lp0 + k;
                     int32_t pg = -1;
                     if (lp < lp_end) {
-                        const int idx = lp - lp_begin;
-                        if (idx < kMaxPageIds) {
-                            pg = s_pages[idx];
+                        if (lp < kMaxPageIds) {
+                            pg = s_pages[lp];
                         } else {
                             pg = a.page_table[(int64_t)b * a.max_pages + lp];
                             if (pg < 0 || pg >= a.num_pages) {
@@ -443,34 +594,60 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp == 2) {
         // ============================================================ bias window producer
         const int ht = lane;                              // 0..31
+        // stage rab[h]/2 and the bucket bounds here rather than before the CTA-wide barrier:
+        // the bounds come from the parameter block, whose divergent reads are serialised, and
+        // the first window is not needed before the first S tile
+        for (int k = ht; k < a.NB; k += 32)
+            s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
+        if (bb.count > 0)
+            for (int k = ht; k <= a.NB; k += 32)
+                s_bounds[k] = bb.v[k];
+        else
+            named_barrier_sync(2, 32 + 256);          // device-evaluated bounds (warps 4-11)
+        __syncwarp();
         const int nb = a.NB;
-        const float lg_scale = a.ln_nmax > 0.0 ? (float)((double)(nb - 1) * 0.6931471805599453 / a.ln_nmax) : 0.f;
+        int top = 1;                                      // largest power of two <= nb
+        while (top * 2 <= nb)
+            top *= 2;
         bool ok = true;
         for (int t = 0; t < n; ++t) {
             const int wb = t & 1;
             if (t >= 2) {
-                ok = ok && mbar_wait(&win_empty[wb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
+                ok = ok && mbar_wait_warp(&win_empty[wb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
                 if (!ok)
                     break;
             }
             const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
             const int32_t dist0 = i0 - tg.j0 + (kTile - 1);       // distance at window index 0
             float* wbuf = win + wb * (kWinBuf / 4);
+            int32_t d[8];
+            int k[8];
+#pragma unroll
+            for (int yy = 0; yy < 8; ++yy)
+                d[yy] = dist0 - (ht + 32 * yy);
+            bucket_search8(s_bounds, nb, top, d, k);
 #pragma unroll
             for (int yy = 0; yy < 8; ++yy) {
                 const int y = ht + 32 * yy;
-                const int32_t d = dist0 - y;
-                const float val = (y <= 2 * kTile - 2 && d >= 0) ? s_rab[bucket_fast(s_bounds, nb, d, lg_scale)] : 0.f;
+                const float r = s_rab[k[yy]];
+                const float val = ((y <= 2 * kTile - 2) & (d[yy] >= 0)) ? r : 0.f;
+                // copy s holds the window shifted by s floats after a 4-float pad, so every
+                // lane stores all four copies without a branch
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    if (y - s >= 0)
-                        wbuf[s * kWinStride + (y - s)] = val;
+                    wbuf[s * kWinStride + kWinPad + (y - s)] = val;
             }
             mbar_arrive(&win_full[wb]);
         }
     } else if (warp >= 4) {
         // ============================================================ pointwise + epilogue
         const int pt = threadIdx.x - 128;                 // 0..255
+        if (bb.count == 0) {
+            // bounds not passed by the host (many buckets): evaluate them for the bias warp
+            for (int k = pt; k <= a.NB; k += 256)
+                s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB));
+            named_barrier_sync(2, 32 + 256);
+        }
         const int wg = (warp - 4) >> 2;                   // key-column half
         const int r = ((warp & 3) << 5) + lane;           // query row in the block (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -481,15 +658,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // the window shifted by s floats, so (y0 - s) is a multiple of 4
         const int y0 = (kTile - 1) - r + 64 * wg;
         const int wsel = y0 & 3;
-        const int woff = wsel * kWinStride + (y0 - wsel);
+        const int woff = wsel * kWinStride + kWinPad + (y0 - wsel);
         bool ok = true;
         for (int t = 0; t < n; ++t) {
             const int vst = t % kVStages;
             const int sb = t & 1;
             const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
-            ok = ok && mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
-            ok = ok && mbar_wait(&win_full[sb], (t >> 1) & 1, abort_flag, tmo);
-            ok = __all_sync(0xffffffffu, ok);
+            ok = ok && mbar_wait_warp(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
+            ok = ok && mbar_wait_warp(&win_full[sb], (t >> 1) & 1, abort_flag, tmo);
             if (!ok)
                 break;
             tc_fence_after();
@@ -520,8 +696,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_arrive(&win_empty[sb]);
             // P buffer sb is free once P V of tile t - 2 completed
             if (t >= 2) {
-                ok = ok && mbar_wait(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
-                ok = __all_sync(0xffffffffu, ok);
+                ok = ok && mbar_wait_warp(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
                 if (!ok)
                     break;
             }
@@ -531,7 +706,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (vz < kTile) {
                 // rows past the valid keys may hold anything (page tails, other users): zero
                 // them so that 0 * NaN cannot reach O
-                ok = ok && mbar_wait(&v_full[vst], (t / kVStages) & 1, abort_flag, tmo);
+                ok = ok && mbar_wait_warp(&v_full[vst], (t / kVStages) & 1, abort_flag, tmo);
                 if (ok) {
                     uint8_t* vt = smem + kOffV + vst * kTileBytes;
                     const int first = vz > 0 ? vz : 0;
@@ -543,6 +718,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     fence_proxy_async_smem();
                 }
             }
+            __syncwarp();                                      // .sync.aligned below
             tmem_wait_st();
             if (ok) {
                 tc_fence_before();
@@ -550,8 +726,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
         // ------------------------------------------------------------ epilogue: O / n_max -> workspace
-        ok = ok && mbar_wait(o_full, 0, abort_flag, tmo);
-        ok = __all_sync(0xffffffffu, ok);
+        // the LayerNorm kernel queued behind this grid may start launching now; it waits for
+        // this grid's completion (and memory flush) before it reads the partial outputs
+        pdl_launch_dependents();
+        ok = ok && mbar_wait_warp(o_full, 0, abort_flag, tmo);
         if (ok) {
             tc_fence_after();
             uint32_t ov[64];
@@ -589,10 +767,15 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bo
                     cudaStream_t stream)
 {
     static bool attr_set[2] = {false, false};
-    const int64_t grid_x = (int64_t)a.splits * a.H * B;
-    if (B <= 0 || grid_x <= 0 || a.qblocks <= 0)
+    if (B <= 0 || a.qblocks <= 0)
         return;
-    dim3 grid((unsigned)grid_x, (unsigned)a.qblocks, 1);
+    // paged: one CTA per piece of the balanced plan; the plan sizes its pieces to fit
+    // max(one per SM, one per (entry, head)) CTAs, and CTAs past the last piece exit at once.
+    // Jagged: (head, user) x query block.
+    const int64_t entries = (int64_t)B * a.qblocks;
+    const int64_t paged_grid = entries * a.H > a.target_ctas ? entries * a.H : a.target_ctas;
+    dim3 grid = paged ? dim3((unsigned)paged_grid, 1, 1)
+                      : dim3((unsigned)((int64_t)a.H * B), (unsigned)a.qblocks, 1);
     if (paged) {
         if (!attr_set[1]) {
             cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

@@ -11,19 +11,30 @@
 namespace hstu {
 
 // ------------------------------------------------------------------ workspace layout
-// [0, 256)            : uint32 status word (HSTU_DEV_* bits), rest reserved
-// [256, ...)          : fp32 partial outputs o[split][token][H][D] of the attention kernels
+// [0, 256)                 : uint32 status word (HSTU_DEV_* bits), rest reserved
+// [256, 256 + C)           : int32 per-token split counts (paged), C = tokens * 4 rounded to 256
+// [256 + C, ...)           : fp32 partial outputs o[split][token][H][D] of the attention kernels
 constexpr size_t kStatusBytes = 256;
-constexpr int kMaxSplits = 16;
+constexpr int kMaxSplits = 8;
+
+__host__ __device__ __forceinline__ size_t counts_bytes(int64_t tokens)
+{
+    return ((size_t)tokens * 4 + 255) & ~(size_t)255;
+}
 
 __device__ __forceinline__ void set_flag(void* ws, uint32_t bits)
 {
     atomicOr(reinterpret_cast<unsigned int*>(ws), bits);
 }
 
-__host__ __device__ __forceinline__ float* partials(void* ws)
+__host__ __device__ __forceinline__ int32_t* split_counts(void* ws)
 {
-    return reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kStatusBytes);
+    return reinterpret_cast<int32_t*>(reinterpret_cast<char*>(ws) + kStatusBytes);
+}
+
+__host__ __device__ __forceinline__ float* partials(void* ws, int64_t tokens)
+{
+    return reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kStatusBytes + counts_bytes(tokens));
 }
 
 // ------------------------------------------------------------------ relative-position bucket

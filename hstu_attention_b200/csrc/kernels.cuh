@@ -15,7 +15,8 @@ struct SimtArgs {
     const int32_t *cached_lens, *new_lens; // paged
     const int32_t* num_targets;
     const float* rab;
-    void* ws;
+    void* ws;                              // status word
+    float* part;                           // fp32 partial outputs [tokens][H][D] (one plane)
     int64_t total_tokens;                  // jagged: all tokens; paged: all new tokens
     int32_t max_len;                       // jagged: max_seqlen; paged: max_new
     int32_t H, D, NB, n_max, P, num_pages, max_pages;
@@ -29,10 +30,15 @@ struct TcArgs {
     const int32_t* num_targets;
     const int32_t* page_table;
     const float* rab;
-    void* ws;
+    void* ws;               // status word
+    float* part;            // fp32 partial outputs [max_splits][tokens][H][D]
+    int32_t* counts;        // paged: per-token number of partial planes written (split count)
     int64_t total_tokens;   // rows of q/k/v/u (jagged) or of the new-token arrays (paged)
     int32_t max_len;        // jagged: max_seqlen; paged: max_new
-    int32_t H, NB, n_max, P, num_pages, max_pages, splits, qblocks;
+    int32_t H, NB, n_max, P, num_pages, max_pages, qblocks;
+    int32_t B;              // users
+    int32_t max_splits;     // paged: partial planes available
+    int32_t target_ctas;    // paged: CTAs the balanced split aims for (one per SM)
     double ln_nmax;
     float inv_n;
     uint64_t timeout_ns;
@@ -57,8 +63,9 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
                       int32_t esize,
                       int32_t P, int32_t num_pages, int32_t max_pages, int32_t max_new, void* ws,
                       cudaStream_t stream);
-void launch_ln_gate(const float* part, int32_t S, int64_t ntok, int32_t HD, const void* u, void* out, bool fp32,
-                    float eps, cudaStream_t stream);
+// counts == nullptr: every token has S partial planes; otherwise token t has counts[t].
+void launch_ln_gate(const float* part, int32_t S, const int32_t* counts, int64_t ntok, int32_t HD, const void* u,
+                    void* out, bool fp32, float eps, cudaStream_t stream);
 void launch_attn_simt(const SimtArgs& a, bool paged, bool fp32, int32_t B, cudaStream_t stream);
 void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
                     cudaStream_t stream);

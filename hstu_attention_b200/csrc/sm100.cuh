@@ -55,8 +55,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the waiting warp sleeps in hardware until the phase
+// completes or about `hint_ns` pass, instead of spinning on issue slots and shared-memory
+// bandwidth that the working warps need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: gives up after `limit_ns` of wall time or once *abort is set by another
 // role of the CTA; on its own timeout it sets *abort.  Returns true when the phase completed.
+// Each poll is a try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes (or ~0.2 ms pass), so a waiting warp neither spins nor oversleeps the way a
+// software sleep would.  The abort flag and the clock are read only between such polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns)
 {
@@ -64,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait(bar, parity))
+        if (mbar_try_wait_sleep(bar, parity, 200000u))
             return true;
         if (*abort)
             return false;
@@ -75,6 +94,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Whole-warp wait: lane 0 polls, the others sleep in __syncwarp; the warp leaves converged
+// and, through __syncwarp's memory ordering, with lane 0's acquire visible to every lane.
+// Polling from one lane instead of 32 keeps the shared-memory pipe free for the warps that
+// are working.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait(bar, parity, abort, limit_ns);
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // ------------------------------------------------------------------ special functions
 // Hardware tanh approximation (one MUFU operation; absolute error about 2^-11).
 __device__ __forceinline__ float tanh_approx(float x)
@@ -82,6 +115,19 @@ __device__ __forceinline__ float tanh_approx(float x)
     float y;
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Allow the grid launched after this one (with programmatic stream serialization) to start.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the grid this one depends on has completed and its memory is visible.
+__device__ __forceinline__ void pdl_wait_primary()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ packed fp32 pairs (sm_100)
@@ -131,6 +177,17 @@ __device__ __forceinline__ void tanh2_f16(float a, float b, float& ta, float& tb
     asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
         : "=f"(ta), "=f"(tb)
         : "r"(t));
+}
+
+// Two fp32 values rounded to bf16 on the integer pipe (add half an ulp of bf16 to the bit
+// pattern, keep the high halves): round-half-away-from-zero, which differs from
+// round-to-nearest-even only on exact ties.  Keeps the conversion off the special-function
+// pipe, which the pointwise SiLU already saturates with tanh.  Finite inputs only.
+__device__ __forceinline__ uint32_t bf16x2_round_int(float lo, float hi)
+{
+    const uint32_t a = __float_as_uint(lo) + 0x8000u;
+    const uint32_t b = __float_as_uint(hi) + 0x8000u;
+    return __byte_perm(a, b, 0x7632);
 }
 
 // ------------------------------------------------------------------ fences
