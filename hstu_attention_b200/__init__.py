@@ -31,6 +31,8 @@ DEV_BAD_NMAX = 1 << 2
 DEV_TIMEOUT = 1 << 3
 DEV_SMEM_ALIGN = 1 << 4
 
+ERR_SCRATCH_LIMIT = -5
+
 EXPORTED = (
     "hstu_version",
     "hstu_error_string",
@@ -39,6 +41,7 @@ EXPORTED = (
     "hstu_read_status",
     "hstu_attn_jagged_fwd",
     "hstu_attn_paged_fwd",
+    "hstu_attn_paged_fwd_noalloc",
     "hstu_kv_append",
     "hstu_bucket_table",
 )
@@ -90,6 +93,9 @@ def load(path: Optional[str] = None):
             lib.hstu_attn_paged_fwd.restype = ctypes.c_int
             lib.hstu_attn_paged_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                 vp, sz, vp]
+            lib.hstu_attn_paged_fwd_noalloc.restype = ctypes.c_int
+            lib.hstu_attn_paged_fwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64,
+                                                        i32, vp, vp]
             lib.hstu_kv_append.restype = ctypes.c_int
             lib.hstu_kv_append.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, sz, vp]
             lib.hstu_bucket_table.restype = ctypes.c_int
@@ -195,6 +201,24 @@ def paged_fwd(p: HstuParams, q_new, k_new, v_new, u_new, k_pages, v_pages, page_
                                     _ptr(new_lens), _ptr(num_targets), _ptr(rab), _ptr(out), B, q_new.shape[0],
                                     int(max_new), workspace.ptr, workspace.nbytes, _stream(stream))
     _check(rc, "hstu_attn_paged_fwd")
+    return out
+
+
+def paged_fwd_noalloc(p: HstuParams, q_new, k_new, v_new, u_new, k_pages, v_pages, page_table, cached_lens,
+                      new_lens, num_targets, rab, *, max_new: int, out=None, flags=None, stream=None):
+    """hstu_attn_paged_fwd_noalloc: paged_fwd on the library's built-in 8 MiB scratch instead of a
+    workspace.  ``flags``: optional 1-element int32 CUDA tensor that receives this call's device
+    status bits.  All calls on a device share the scratch: do not overlap them across streams."""
+    import torch
+
+    if out is None:
+        out = torch.empty_like(q_new)
+    B = cached_lens.shape[0]
+    rc = load().hstu_attn_paged_fwd_noalloc(ctypes.byref(p), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(u_new),
+                                            _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(cached_lens),
+                                            _ptr(new_lens), _ptr(num_targets), _ptr(rab), _ptr(out), B,
+                                            q_new.shape[0], int(max_new), _ptr(flags), _stream(stream))
+    _check(rc, "hstu_attn_paged_fwd_noalloc")
     return out
 
 

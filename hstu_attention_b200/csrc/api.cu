@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points declared in include/hstu.h: argument validation,
 // workspace accounting, TMA descriptor encoding and kernel dispatch.
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -201,6 +202,39 @@ static int finish(cudaStream_t)
 
 static constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s per in-kernel wait
 
+// Scratch of hstu_attn_paged_fwd_noalloc: a fixed array in the library's own device image, so
+// that callers which cannot hand over a workspace still get a paged forward.  Layout is the
+// workspace layout (status block, split counts, fp32 partial planes).  Every call on a device
+// shares it.
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+static std::atomic<void*> g_noalloc_ptr[kNoAllocMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device, looked up on the first call per
+// device (the lookup may load this library's device code onto that device).
+static int noalloc_scratch(void** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    if (dev >= 0 && dev < kNoAllocMaxDevices) {
+        void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+        if (p) {
+            *out = p;
+            return HSTU_OK;
+        }
+    }
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+        return HSTU_ERR_CUDA;
+    if (dev >= 0 && dev < kNoAllocMaxDevices)
+        g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    *out = p;
+    return HSTU_OK;
+}
+
 }  // namespace hstu
 
 using namespace hstu;
@@ -217,6 +251,8 @@ const char* hstu_error_string(int code)
     case HSTU_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case HSTU_ERR_WORKSPACE: return "workspace too small or misaligned";
     case HSTU_ERR_CUDA: return "CUDA error";
+    case HSTU_ERR_SCRATCH_LIMIT:
+        return "request needs more than the 8 MiB built-in scratch of hstu_attn_paged_fwd_noalloc";
     default: return "unknown error";
     }
 }
@@ -472,6 +508,44 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
     launch_ln_gate(part, splits, use_tc(params) ? counts : nullptr, total_new, params->num_heads * params->head_dim,
                    u_new, out, fp32, params->ln_eps, s);
     return finish(s);
+}
+
+
+int hstu_attn_paged_fwd_noalloc(const hstu_attn_params* params, const void* q_new, const void* k_new,
+                                const void* v_new, const void* u_new, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, const int32_t* cached_lens, const int32_t* new_lens,
+                                const int32_t* num_targets, const float* rab, void* out, int32_t B,
+                                int64_t total_new, int32_t max_new, uint32_t* flags_out, void* stream)
+{
+    int rc = check_params(params, true);
+    if (rc != HSTU_OK)
+        return rc;
+    if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
+        return HSTU_ERR_INVALID_ARG;
+    if (flags_out && (reinterpret_cast<uintptr_t>(flags_out) & 3u))
+        return HSTU_ERR_INVALID_ARG;
+    // the status block, the split counts and at least one partial plane must fit; more room
+    // only buys more key splits
+    const size_t need = kStatusBytes + counts_bytes(total_new) + partial_bytes(params, 1, total_new);
+    if (need > kNoAllocScratchBytes)
+        return HSTU_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc != HSTU_OK)
+        return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the status word is the only part that must start at zero: cleared for every call
+    if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    rc = hstu_attn_paged_fwd(params, q_new, k_new, v_new, u_new, k_pages, v_pages, page_table, cached_lens,
+                             new_lens, num_targets, rab, out, B, total_new, max_new, scratch, kNoAllocScratchBytes,
+                             stream);
+    if (rc != HSTU_OK)
+        return rc;
+    if (flags_out &&
+        cudaMemcpyAsync(flags_out, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    return HSTU_OK;
 }
 
 }  // extern "C"

@@ -57,7 +57,9 @@ typedef enum {
     HSTU_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misaligned pointer */
     HSTU_ERR_UNSUPPORTED = -2,  /* a shape this build does not implement */
     HSTU_ERR_WORKSPACE = -3,    /* workspace too small or misaligned */
-    HSTU_ERR_CUDA = -4          /* a CUDA runtime/driver call failed */
+    HSTU_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed */
+    HSTU_ERR_SCRATCH_LIMIT = -5 /* hstu_attn_paged_fwd_noalloc: the request does not fit the
+                                   library's built-in 8 MiB scratch */
 } hstu_status_code;
 
 typedef enum { HSTU_DTYPE_BF16 = 0, HSTU_DTYPE_FP32 = 1 } hstu_dtype;
@@ -151,6 +153,43 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
                         const int32_t* num_targets, const float* rab, void* out, int32_t B,
                         int64_t total_new, int32_t max_new, void* workspace,
                         size_t workspace_bytes, void* stream);
+
+/*
+ * hstu_attn_paged_fwd without a workspace argument.  The pages describe no such call: it is
+ * a convenience of this library for callers that cannot allocate device memory or keep a
+ * buffer of their own across calls -- for example an operator plugin inside a host runtime
+ * that owns all device allocations, or code on a path where allocating would stall or
+ * fragment a memory pool.
+ *
+ * Arguments are those of hstu_attn_paged_fwd, with the workspace pair replaced by
+ *   flags_out : optional DEVICE pointer (4-byte aligned) that receives, in stream order, the
+ *               HSTU_DEV_* bits this call raised (0 = clean); NULL skips the copy.
+ *
+ * Scratch: a fixed 8 MiB array (8,388,608 bytes) compiled into the library, one per device,
+ * laid out like a workspace.  Nothing is allocated: no cudaMalloc, cudaFree or allocating
+ * library routine is called.  A request needs 256 + 4*total_new (rounded up to 256) +
+ * 4*total_new*H*D bytes for one fp32 partial plane; if that exceeds 8 MiB the call returns
+ * HSTU_ERR_SCRATCH_LIMIT and launches nothing (at H*D = 512 that is total_new > 4087).  Spare
+ * room holds further partial planes, so the key range may be split over fewer CTAs than
+ * with a full workspace; results agree with hstu_attn_paged_fwd up to fp32 summation order.
+ *
+ * Of the scratch, only the status word must start at zero; each call clears it on `stream`
+ * before its kernels run.  All calls on one device share the array, so two calls that may
+ * run concurrently (different streams, different host threads) race and corrupt each
+ * other's results: order them on one stream, or use hstu_attn_paged_fwd with separate
+ * workspaces.
+ *
+ * The first call on each device does a one-time set-up: it looks up the array's device
+ * address (cudaGetSymbolAddress on the current device), which may load the library's device
+ * code onto that device.  Make that first call before any stream capture begins.
+ */
+int hstu_attn_paged_fwd_noalloc(const hstu_attn_params* params, const void* q_new,
+                                const void* k_new, const void* v_new, const void* u_new,
+                                const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, const int32_t* cached_lens,
+                                const int32_t* new_lens, const int32_t* num_targets,
+                                const float* rab, void* out, int32_t B, int64_t total_new,
+                                int32_t max_new, uint32_t* flags_out, void* stream);
 
 /*
  * Append new history tokens into the pages (the KV cache's "append"; NVIDIA blog, section
