@@ -70,7 +70,9 @@ constexpr uint32_t kSmemBytes = kSmemUsed + 1024;     // slack to align the base
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
 
+constexpr uint32_t kOStride = kTcD + 4;       // floats per row of the staged O tile (epilogue)
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffK + kTile * kOStride * 4 <= kOffWin, "epilogue staging fits the K and V rings");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 
 struct TileGeo {
@@ -194,9 +196,14 @@ struct PlanTiles {
     int t[kPlanRounds];
 };
 
+// min(ceil(t / c), max_splits) for t >= 0, by comparisons (no integer division).
 __device__ __forceinline__ int splits_for(int t, int c, int max_splits)
 {
-    return t == 0 ? 0 : min((t + c - 1) / c, max_splits);
+    int s = 0;
+#pragma unroll
+    for (int k = 0; k < kMaxSplits; ++k)
+        s += ((k < max_splits) & (t > k * c)) ? 1 : 0;
+    return s;
 }
 
 // Tiles per piece c: start from ceil(all tiles over all heads / target_ctas) and grow until
@@ -730,6 +737,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // this grid's completion (and memory flush) before it reads the partial outputs
         pdl_launch_dependents();
         ok = ok && mbar_wait_warp(o_full, 0, abort_flag, tmo);
+        // every MMA has completed, so the K and V rings are free: O (scaled by 1/n_max) goes
+        // row by row into a padded fp32 tile there, then each warp writes whole rows (512
+        // contiguous bytes per instruction) instead of one 16-byte piece per row
+        float* ostage = reinterpret_cast<float*>(smem + kOffK);
         if (ok) {
             tc_fence_after();
             uint32_t ov[64];
@@ -737,14 +748,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_ld_32x32b_x32(ocol, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
             tmem_ld_32x32b_x32(ocol + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
             tmem_wait_ld();
-            if (row_valid) {
-                const float inv_n = a.inv_n;
-                float4* dst = reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + r) * HD + (int64_t)h * kTcD + wg * 64);
+            const float inv_n = a.inv_n;
+            float4* srow = reinterpret_cast<float4*>(ostage + r * kOStride + wg * 64);
 #pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4)
-                    dst[c4] = make_float4(__uint_as_float(ov[4 * c4]) * inv_n, __uint_as_float(ov[4 * c4 + 1]) * inv_n,
-                                          __uint_as_float(ov[4 * c4 + 2]) * inv_n,
-                                          __uint_as_float(ov[4 * c4 + 3]) * inv_n);
+            for (int c4 = 0; c4 < 16; ++c4)
+                srow[c4] = make_float4(__uint_as_float(ov[4 * c4]) * inv_n, __uint_as_float(ov[4 * c4 + 1]) * inv_n,
+                                       __uint_as_float(ov[4 * c4 + 2]) * inv_n,
+                                       __uint_as_float(ov[4 * c4 + 3]) * inv_n);
+        }
+        named_barrier_sync(3, 256);                           // the eight pointwise warps
+        if (ok) {
+            const int pw = pt >> 5;                           // 0..7
+            const int nrows = min(kTile, g.N - qrow0);
+            for (int row = pw; row < nrows; row += 8) {
+                const float4 v = reinterpret_cast<const float4*>(ostage + row * kOStride)[lane];
+                reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + row) * HD + (int64_t)h * kTcD)[lane] = v;
             }
         }
     }

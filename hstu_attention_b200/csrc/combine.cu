@@ -17,7 +17,7 @@
 
 namespace hstu {
 
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 128;   // small blocks fit beside a resident attention CTA
 
 template <typename T> struct Vec4;
 template <> struct Vec4<float> {
