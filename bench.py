@@ -46,6 +46,28 @@ def load_peaks():
         return PEAKS_FALLBACK, "fallback"
 
 
+# ----------------------------------------------------------------------------- replicas
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest of every rank's x (the job time of weak-scaled replicas); x itself when the
+    process group is not initialised.  NCCL ranks pass their CUDA device, gloo ranks the CPU."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, ms_per_step: float, world: int) -> float:
+    """Whole-job units/s of `world` replicas that each process units_per_rank_step per step,
+    with ms_per_step the max over ranks."""
+    return units_per_rank_step * world / (ms_per_step * 1e-3)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -405,13 +427,11 @@ def main():
     # per-call durations of the last replay's paged attention calls
     for a, b in events:
         call_ms.append(a.elapsed_time(b))
+    elapsed_ms = max_over_ranks(elapsed_ms, device)
     if world > 1:
-        t = torch.tensor([elapsed_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
         dist.barrier()
     ms_step = elapsed_ms / args.steps
-    value = tokens * world / (ms_step * 1e-3)
+    value = job_throughput(tokens, ms_step, world)
     assert ws.status() == 0, "device status flags set during the timed region"
 
     # e2e through the public API with host buffers: per step, H2D of every layer's new-token
@@ -443,11 +463,7 @@ def main():
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e_steps, device)
 
     prefill = None
     if rank == 0 and not args.no_prefill:
@@ -494,7 +510,7 @@ def main():
                      "ms_per_call": mean_call_ms,
                      "tflops": float(np.mean(lflops)) / (mean_call_ms * 1e-3) / 1e12},
         "cpu_baseline": cpu,
-        "e2e": {"value": tokens * world / (e2e_ms * 1e-3), "unit": "new tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(tokens, e2e_ms, world), "unit": "new tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 3 * len(L),
         "clocks": clocks,
