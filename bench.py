@@ -33,6 +33,26 @@ sys.path.insert(0, ROOT)
 from hstu_attention_b200 import inputs as gen  # noqa: E402
 
 METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline"
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per paged call on one layer of this
+# batch, from one `ncu --set full` capture (profiles/attn_tc_paged_cachehit_layer0.md):
+# attn_tc_kernel 41.923 MB + 6.1 KB, ln_gate_kernel 6.571 MB (ncu flushes caches, so the
+# LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for the kernel
+# sources they were taken from (hash below); otherwise the bench reports traffic as null.
+PAGED_TRAFFIC_BYTES = 41.923328e6 + 6.144e3 + 6.571264e6
+PAGED_TRAFFIC_SOURCES = "f9e85f47b1a3c330"
+# the same capture for the jagged prefill attention kernel (profiles/attn_tc_jagged_prefill_8users.md)
+PREFILL_TRAFFIC_BYTES = 63.617536e6 + 10.822912e6
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("attn_tc.cu", "combine.cu"):
+        with open(os.path.join(ROOT, "hstu_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -267,7 +287,8 @@ def bench_prefill(hb, device, steps, warmup, peaks):
     return {"workload": "jagged prefill: 8 users, lengths U[256,4096] (seed 1002), 64 candidates, H=4, D=128",
             "tokens": int(c.T), "ms_per_call": ms, "tokens_per_s": c.T / (ms * 1e-3), "tflops": tf,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                         "traffic": None},
+                         "traffic": PREFILL_TRAFFIC_BYTES if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None,
+                         "traffic_kernel": "attn_tc_kernel (jagged) per launch"},
             "launches_per_call": 2}
 
 
@@ -505,7 +526,8 @@ def main():
                    "graph": "one CUDA graph per step; appends on a forked stream (they do not feed "
                             "the attention, which reads new keys from k_new)"},
         "roofline": {"bound": "hbm", "kernel": "hstu_attn_paged_fwd (attention kernel + LayerNorm-gate kernel)",
-                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": PAGED_TRAFFIC_BYTES if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None,
                      "peak_kind": peaks_kind, "algorithmic_bytes_per_call": mean_bytes,
                      "ms_per_call": mean_call_ms,
                      "tflops": float(np.mean(lflops)) / (mean_call_ms * 1e-3) / 1e12},
