@@ -33,6 +33,8 @@ DEV_SMEM_ALIGN = 1 << 4
 
 ERR_SCRATCH_LIMIT = -5
 
+FLAG_OVERLAP_PREVIOUS = 1 << 0
+
 EXPORTED = (
     "hstu_version",
     "hstu_error_string",
@@ -60,6 +62,7 @@ class HstuParams(ctypes.Structure):
         ("num_pages", ctypes.c_int32),
         ("max_pages_per_user", ctypes.c_int32),
         ("ln_eps", ctypes.c_float),
+        ("flags", ctypes.c_uint32),
     ]
 
 
@@ -115,7 +118,7 @@ def _check(rc: int, what: str):
 
 
 def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, page_size: int = 0,
-           num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5) -> HstuParams:
+           num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5, flags: int = 0) -> HstuParams:
     import torch
 
     if dtype in (torch.bfloat16, "bf16"):
@@ -125,7 +128,7 @@ def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, p
     else:
         raise HstuError(f"unsupported dtype {dtype}")
     return HstuParams(num_heads, head_dim, dt, num_buckets, n_max, page_size, num_pages, max_pages_per_user,
-                      ln_eps)
+                      ln_eps, flags)
 
 
 def _ptr(t) -> Optional[int]:

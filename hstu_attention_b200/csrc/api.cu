@@ -100,6 +100,8 @@ static int check_params(const hstu_attn_params* p, bool paged)
         return HSTU_ERR_INVALID_ARG;
     if (!(p->ln_eps >= 0.0f) || !isfinite(p->ln_eps))
         return HSTU_ERR_INVALID_ARG;
+    if (p->flags & ~(uint32_t)HSTU_FLAG_OVERLAP_PREVIOUS)
+        return HSTU_ERR_INVALID_ARG;
     if (p->dtype != HSTU_DTYPE_BF16 && p->dtype != HSTU_DTYPE_FP32)
         return HSTU_ERR_UNSUPPORTED;
     if (p->head_dim != 32 && p->head_dim != 64 && p->head_dim != 128)
@@ -478,6 +480,7 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.timeout_ns = kTimeoutNs;
+        a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
         launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), true, B, s);
     } else {
         SimtArgs a{};

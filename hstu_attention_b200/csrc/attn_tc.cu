@@ -373,14 +373,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int32_t n = g.ok ? t_end - t_begin : 0;
     const int64_t HD = (int64_t)a.H * kTcD;
     float* part = a.part + (int64_t)split * a.total_tokens * HD;
-    if (kPaged && h == 0 && split == 0) {
-        // the LayerNorm kernel sums this many partial planes for each of these tokens
-        for (int r = threadIdx.x; r < kTile; r += kTcThreads)
-            if (qrow0 + r < g.N)
-                a.counts[g.tok0 + qrow0 + r] = g.ok ? nsplit : 1;
-    }
+    // the LayerNorm kernel sums this many partial planes for each of these tokens (written once
+    // the kernel before this one -- possibly the previous call's LayerNorm kernel, which reads
+    // the same workspace -- has finished)
+    auto write_counts = [&]() {
+        if (kPaged && h == 0 && split == 0)
+            for (int r = threadIdx.x; r < kTile; r += kTcThreads)
+                if (qrow0 + r < g.N)
+                    a.counts[g.tok0 + qrow0 + r] = g.ok ? nsplit : 1;
+    };
 
     if (n <= 0) {
+        pdl_wait_primary();
+        write_counts();
         // nothing to accumulate: this split's partial rows are zero
         for (int x = threadIdx.x; x < kTile * (kTcD / 4); x += kTcThreads) {
             const int r = x / (kTcD / 4), c4 = x % (kTcD / 4);
@@ -466,6 +471,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = a.timeout_ns;
+    // everything above only read the length arrays and the page table; inputs and the workspace
+    // are touched only after the previous kernel on the stream has finished (a no-op unless
+    // this grid was launched as a programmatic dependent)
+    pdl_wait_primary();
+    write_counts();
 
     if ((warp == 0 || warp == 3) && lane == 0) {
         // ============================================================ TMA producers
@@ -799,7 +809,21 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bo
             cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
             attr_set[1] = true;
         }
-        attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
+        if (a.overlap_previous) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = grid;
+            cfg.blockDim = dim3(kTcThreads, 1, 1);
+            cfg.dynamicSmemBytes = kSmemBytes;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
+        } else {
+            attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
+        }
     } else {
         if (!attr_set[0]) {
             cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);

@@ -42,6 +42,7 @@ struct TcArgs {
     double ln_nmax;
     float inv_n;
     uint64_t timeout_ns;
+    int32_t overlap_previous;   // paged: launched as a programmatic dependent of the previous kernel
 };
 
 struct TcMaps {

@@ -375,3 +375,37 @@ def test_mixed_batch_sampled(cuda_lib):
             page = int(miss_pt[b, pos // 32])
             got = host(kp[page, :, pos % 32, :])
             assert np.array_equal(got, misses.k[s0 + pos])
+
+
+# --------------------------------------------------------------------------- launch overlap flag
+
+
+def test_overlap_previous_flag_is_bit_identical(cuda_lib):
+    """HSTU_FLAG_OVERLAP_PREVIOUS only changes when the kernel may start: back-to-back paged calls
+    sharing one workspace (each call's set-up overlapping the previous call's LayerNorm kernel)
+    give the same bytes as calls without the flag."""
+    import torch
+
+    hb = cuda_lib
+    cases = [_paged_small(32, seed=s) for s in (101, 102, 103)]
+    c0 = cases[0]
+    pools = [device_pool(c) for c in cases]
+
+    def run(flags):
+        p = hb.params(c0.H, c0.D, c0.dtype, c0.NB, c0.n_max, page_size=c0.P, num_pages=c0.num_pages,
+                      max_pages_per_user=c0.max_pages, ln_eps=c0.eps, flags=flags)
+        ws = hb.Workspace(p, c0.B, max(c.Tn for c in cases), max(c.max_new for c in cases))
+        outs = []
+        for _ in range(2):
+            for c, (kp, vp) in zip(cases, pools):
+                outs.append(hb.paged_fwd(p, dev(c.q_new), dev(c.k_new), dev(c.v_new), dev(c.u_new), kp, vp,
+                                         dev(c.page_table), dev(c.cached_lens), dev(c.new_lens), dev(c.num_targets),
+                                         dev(c.rab), max_new=c.max_new, workspace=ws))
+        torch.cuda.synchronize()
+        assert ws.status() == 0
+        return outs
+
+    plain, overlapped = run(0), run(hb.FLAG_OVERLAP_PREVIOUS)
+    for a, b in zip(plain, overlapped):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert_close(host(overlapped[0]), oracle_paged(cases[0]), "bf16", "overlapped call vs oracle")
