@@ -36,13 +36,13 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per paged call on one layer of this
 # batch, from one `ncu --set full` capture (profiles/attn_tc_paged_cachehit_layer0.md):
-# attn_tc_kernel 41.923 MB + 6.1 KB, ln_gate_kernel 6.571 MB (ncu flushes caches, so the
+# attn_tc_kernel 41.924 MB + 2.3 KB, ln_gate_kernel 6.571 MB (ncu flushes caches, so the
 # LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for the kernel
 # sources they were taken from (hash below); otherwise the bench reports traffic as null.
-PAGED_TRAFFIC_BYTES = 41.923328e6 + 6.144e3 + 6.571264e6
-PAGED_TRAFFIC_SOURCES = "f9e85f47b1a3c330"
+PAGED_TRAFFIC_BYTES = 41.923584e6 + 2.304e3 + 6.570752e6
+PAGED_TRAFFIC_SOURCES = "34d0063844333004"
 # the same capture for the jagged prefill attention kernel (profiles/attn_tc_jagged_prefill_8users.md)
-PREFILL_TRAFFIC_BYTES = 63.617536e6 + 10.822912e6
+PREFILL_TRAFFIC_BYTES = 63.182592e6 + 11.64672e6
 
 
 def kernel_sources_hash() -> str:

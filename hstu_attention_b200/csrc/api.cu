@@ -130,18 +130,20 @@ static bool use_tc(const hstu_attn_params* p)
     return p->dtype == HSTU_DTYPE_BF16 && p->head_dim == 128 && p->num_buckets <= 1024;
 }
 
+// SM count of the current device (cached per device; 148 if the query fails).
 static int num_sms()
 {
-    static int cached = 0;
-    if (cached == 0) {
-        int dev = 0, n = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
-            cached = n;
-        else
-            return 148;
-    }
-    return cached;
+    static std::atomic<int> cached[64];
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 148;
+    if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0)
+        return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    if (dev >= 0 && dev < 64)
+        cached[dev].store(n, std::memory_order_relaxed);
+    return n;
 }
 
 static size_t partial_bytes(const hstu_attn_params* p, int splits, int64_t tokens)

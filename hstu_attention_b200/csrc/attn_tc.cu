@@ -36,6 +36,8 @@
 //   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 2 bias windows | bucket bounds | rab | page ids |
 //   mbarriers
 // Every wait is bounded (HSTU_DEV_TIMEOUT) so a logic error cannot hang the GPU.
+#include <atomic>
+
 #include "common.cuh"
 #include "sm100.cuh"
 #include "kernels.cuh"
@@ -794,9 +796,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
                     cudaStream_t stream)
 {
-    static bool attr_set[2] = {false, false};
     if (B <= 0 || a.qblocks <= 0)
         return;
+    // the shared-memory opt-in is a per-device setting of each kernel
+    static std::atomic<uint32_t> attr_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint32_t bit = paged ? 2u : 1u;
+    if (dev < 0 || dev >= 64 || !(attr_set[dev].load(std::memory_order_relaxed) & bit)) {
+        if (paged)
+            cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        else
+            cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (dev >= 0 && dev < 64)
+            attr_set[dev].fetch_or(bit, std::memory_order_relaxed);
+    }
     // paged: one CTA per piece of the balanced plan; the plan sizes its pieces to fit
     // max(one per SM, one per (entry, head)) CTAs, and CTAs past the last piece exit at once.
     // Jagged: (head, user) x query block.
@@ -805,10 +819,6 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bo
     dim3 grid = paged ? dim3((unsigned)paged_grid, 1, 1)
                       : dim3((unsigned)((int64_t)a.H * B), (unsigned)a.qblocks, 1);
     if (paged) {
-        if (!attr_set[1]) {
-            cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-            attr_set[1] = true;
-        }
         if (a.overlap_previous) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = grid;
@@ -825,10 +835,6 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bo
             attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
         }
     } else {
-        if (!attr_set[0]) {
-            cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-            attr_set[0] = true;
-        }
         attn_tc_kernel<false><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
     }
 }
