@@ -100,3 +100,22 @@ def test_host_validation_without_gpu(lib):
     bad_ws[-3] = None
     assert A(ctypes.byref(p), *bad_ws) == -3
     assert lib.hstu_bucket_table(ctypes.byref(p), -1, None, None) == -1
+
+
+def test_flags_and_noalloc_limit_without_gpu(lib):
+    """Unknown flag bits are rejected; the allocation-free entry rejects a request larger than its
+    built-in 8 MiB scratch before it touches the device."""
+    bad = _p(flags=1 << 7)
+    assert lib.hstu_workspace_size(ctypes.byref(bad), 1, 1, 1) == 0
+    ok = _p(flags=hb.FLAG_OVERLAP_PREVIOUS)
+    assert lib.hstu_workspace_size(ctypes.byref(ok), 1, 1, 1) > 0
+    fake = 1 << 20
+    N = lib.hstu_attn_paged_fwd_noalloc
+    # 4,088 new tokens at H*D = 512 need 256 + 16,384 + 8,372,224 bytes > 8 MiB
+    args = [fake] * 6 + [fake, fake, fake, None, fake, fake, 1, 4088, 4088, None, None]
+    assert N(ctypes.byref(_p(n_max=8192)), *args) == hb.ERR_SCRATCH_LIMIT
+    assert "8 MiB" in lib.hstu_error_string(hb.ERR_SCRATCH_LIMIT).decode()
+    assert N(ctypes.byref(bad), *args) == -1
+    misaligned_flags = list(args)
+    misaligned_flags[-2] = fake + 2                                       # flags_out not 4-byte aligned
+    assert N(ctypes.byref(_p(n_max=8192)), *misaligned_flags) == -1
