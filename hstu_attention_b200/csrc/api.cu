@@ -388,6 +388,7 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.timeout_ns = kTimeoutNs;
+        a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
         launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), false, B, s);
     } else {
         SimtArgs a{};

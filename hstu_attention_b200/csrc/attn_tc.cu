@@ -818,25 +818,20 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bo
     const int64_t paged_grid = entries * a.H > a.target_ctas ? entries * a.H : a.target_ctas;
     dim3 grid = paged ? dim3((unsigned)paged_grid, 1, 1)
                       : dim3((unsigned)((int64_t)a.H * B), (unsigned)a.qblocks, 1);
-    if (paged) {
-        if (a.overlap_previous) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = grid;
-            cfg.blockDim = dim3(kTcThreads, 1, 1);
-            cfg.dynamicSmemBytes = kSmemBytes;
-            cfg.stream = stream;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[0].val.programmaticStreamSerializationAllowed = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
-        } else {
-            attn_tc_kernel<true><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
-        }
-    } else {
-        attn_tc_kernel<false><<<grid, kTcThreads, kSmemBytes, stream>>>(m.q, m.k, m.v, m.kp, m.vp, bb, a);
-    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.overlap_previous ? 1 : 0;          // programmatic dependent launch on request
+    if (paged)
+        cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
+    else
+        cudaLaunchKernelEx(&cfg, attn_tc_kernel<false>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
 }
 
 }  // namespace hstu

@@ -92,16 +92,16 @@ typedef struct {
 /*
  * Bits of hstu_attn_params.flags.
  *
- * HSTU_FLAG_OVERLAP_PREVIOUS (paged calls): the attention kernel is launched with programmatic
- * dependent launch, so its set-up -- the work plan from cached_lens / new_lens / num_targets,
- * the page-table reads, barrier and tensor-memory set-up -- may run while the kernel enqueued
- * before it on the same stream is still finishing.  It waits for that kernel before it reads
- * q/k/v/u, the pages or rab and before it writes anything but the status word.  Set the bit
- * only when the kernel enqueued right before the call does not write page_table, cached_lens,
- * new_lens or num_targets (for example when consecutive layers run back to back, or when the
- * metadata was copied from the host).  Without the bit the call starts after everything before
- * it on the stream has finished.  This is a scheduling choice of this library; the pages
- * describe no such thing.
+ * HSTU_FLAG_OVERLAP_PREVIOUS (attention calls on the tensor-core path): the attention kernel is
+ * launched with programmatic dependent launch, so its set-up -- the work plan from the length
+ * arrays, the page-table reads, barrier and tensor-memory set-up -- may run while the kernel
+ * enqueued before it on the same stream is still finishing.  It waits for that kernel before it
+ * reads q/k/v/u, the pages or rab and before it writes anything but the status word.  Set the
+ * bit only when the kernel enqueued right before the call does not write seq_offsets,
+ * page_table, cached_lens, new_lens or num_targets (for example when consecutive layers run back
+ * to back, or when the metadata was copied from the host).  Without the bit the call starts
+ * after everything before it on the stream has finished.  This is a scheduling choice of this
+ * library; the pages describe no such thing.
  */
 enum { HSTU_FLAG_OVERLAP_PREVIOUS = 1u << 0 };
 

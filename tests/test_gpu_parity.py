@@ -409,3 +409,19 @@ def test_overlap_previous_flag_is_bit_identical(cuda_lib):
     for a, b in zip(plain, overlapped):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert_close(host(overlapped[0]), oracle_paged(cases[0]), "bf16", "overlapped call vs oracle")
+
+    # jagged prefill calls back to back on one workspace
+    jcs = [gen.jagged_case([300, 5, 129], [64, 1, 8], H=4, D=128, NB=128, n_max=512, dtype="bf16", seed=s)
+           for s in (111, 112)]
+
+    def run_j(flags):
+        p = hb.params(4, 128, torch.bfloat16, 128, 512, flags=flags)
+        ws = hb.Workspace(p, 3, max(c.T for c in jcs), 512)
+        outs = [hb.jagged_fwd(p, dev(c.q), dev(c.k), dev(c.v), dev(c.u), dev(c.seq_offsets), dev(c.num_targets),
+                              dev(c.rab), max_seqlen=512, workspace=ws) for _ in range(2) for c in jcs]
+        torch.cuda.synchronize()
+        assert ws.status() == 0
+        return outs
+
+    for a, b in zip(run_j(0), run_j(hb.FLAG_OVERLAP_PREVIOUS)):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
