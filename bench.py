@@ -470,76 +470,95 @@ def main():
     del graph_ev
 
     # e2e through the public API with host buffers: per step, H2D of every layer's new-token
-    # q/k/v/u and metadata from pinned memory, the step, and D2H of every layer's output.  The
-    # layers are pipelined: layer l's upload (copy stream) overlaps layer l-1's kernels (one
-    # small graph per layer) and layer l's download (a second copy stream) overlaps layer l+1.
-    # each layer's inputs live in one pinned host buffer and one device buffer (256-byte aligned
-    # views), so a layer uploads with a single copy
+    # q/k/v/u and metadata from pinned memory, the step, and D2H of every layer's output.  Each
+    # layer's inputs live in one pinned host buffer and one device buffer (256-byte aligned
+    # views), so a layer uploads with a single copy.  Layers are pipelined (layer l's upload on
+    # one copy stream overlaps layer l-1's kernels, one small graph per layer; its download on a
+    # second copy stream overlaps layer l+1), and steps are double-buffered: step s+1 uploads into
+    # the other set of device buffers while step s computes.
     names = ("q", "k", "v", "u", "pt", "cl", "nl", "nt")
-    host_in, dev_in, L_e2e = [], [], []
+    nsets = 2
+    host_in, dev_in, L_e2e = [], [[] for _ in range(nsets)], [[] for _ in range(nsets)]
     for t in L:
         offs, total = [], 0
         for k in names:
             offs.append(total)
             total += (t[k].numel() * t[k].element_size() + 255) // 256 * 256
-        dbuf = torch.empty(total, dtype=torch.uint8, device=device)
         hbuf = torch.empty(total, dtype=torch.uint8).pin_memory()
-        t2 = dict(t)
-        t2["out"] = torch.empty_like(t["out"])
         for k, o in zip(names, offs):
             n = t[k].numel() * t[k].element_size()
-            t2[k] = dbuf[o:o + n].view(t[k].dtype).view(t[k].shape)
             hbuf[o:o + n].copy_(t[k].contiguous().view(torch.uint8).view(-1).cpu())
         host_in.append(hbuf)
-        dev_in.append(dbuf)
-        L_e2e.append(t2)
-    host_out = [t["out"].cpu().pin_memory() for t in L_e2e]
+        for si in range(nsets):
+            dbuf = torch.empty(total, dtype=torch.uint8, device=device)
+            t2 = dict(t)
+            t2["out"] = torch.empty_like(t["out"])
+            for k, o in zip(names, offs):
+                n = t[k].numel() * t[k].element_size()
+                t2[k] = dbuf[o:o + n].view(t[k].dtype).view(t[k].shape)
+            dev_in[si].append(dbuf)
+            L_e2e[si].append(t2)
+    host_out = [[t["out"].cpu().pin_memory() for t in L_e2e[si]] for si in range(nsets)]
     h2d = sum(x.numel() for x in host_in)
-    d2h = sum(x.numel() * x.element_size() for x in host_out)
-    e_steps = max(3, args.steps // 5)
-    layer_graphs = []
-    for t in L_e2e:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            run_step(hb, p, ws, kp, vp, [t], max_new, side=side)
-        layer_graphs.append(g)
+    d2h = sum(x.numel() * x.element_size() for x in host_out[0])
+    e_steps = max(4, args.steps // 5)
+    layer_graphs = [[] for _ in range(nsets)]
+    for si in range(nsets):
+        for t in L_e2e[si]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_step(hb, p, ws, kp, vp, [t], max_new, side=side)
+            layer_graphs[si].append(g)
     up = torch.cuda.Stream(device=device)
     down = torch.cuda.Stream(device=device)
-    ev_up = [torch.cuda.Event() for _ in L]
-    ev_done = [torch.cuda.Event() for _ in L]
+    ev_up = [[torch.cuda.Event() for _ in L] for _ in range(nsets)]
+    ev_done = [[torch.cuda.Event() for _ in L] for _ in range(nsets)]
+    ev_computed = [torch.cuda.Event() for _ in range(nsets)]     # a step's kernels on set si done
+    ev_fetched = [torch.cuda.Event() for _ in range(nsets)]      # a step's downloads from set si done
+    for si in range(nsets):
+        ev_computed[si].record(stream)
+        ev_fetched[si].record(down)
 
-    def e2e_step():
-        up.wait_stream(stream)                  # the previous step has consumed every input
+    def e2e_step(step):
+        si = step % nsets
+        # the step that last used this set has consumed its inputs and shipped its outputs
+        up.wait_event(ev_computed[si])
+        up.wait_event(ev_fetched[si])
         with torch.cuda.stream(up):
-            for li in range(len(L_e2e)):
-                dev_in[li].copy_(host_in[li], non_blocking=True)
-                ev_up[li].record(up)
-        for li, (t, hdst) in enumerate(zip(L_e2e, host_out)):
-            stream.wait_event(ev_up[li])
-            layer_graphs[li].replay()
-            ev_done[li].record(stream)
+            for li in range(len(L)):
+                dev_in[si][li].copy_(host_in[li], non_blocking=True)
+                ev_up[si][li].record(up)
+        for li, t in enumerate(L_e2e[si]):
+            stream.wait_event(ev_up[si][li])
+            layer_graphs[si][li].replay()
+            ev_done[si][li].record(stream)
             with torch.cuda.stream(down):
-                down.wait_event(ev_done[li])
-                hdst.copy_(t["out"], non_blocking=True)
-        stream.wait_stream(down)                # the step ends with its results on the host
+                down.wait_event(ev_done[si][li])
+                host_out[si][li].copy_(t["out"], non_blocking=True)
+        ev_computed[si].record(stream)
+        ev_fetched[si].record(down)
 
-    for _ in range(2):
-        e2e_step()
+    for s_ in range(2):
+        e2e_step(s_)
+    stream.wait_stream(down)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
+    up.wait_stream(stream)                      # the first upload starts after the start event
+    for s_ in range(e_steps):
+        e2e_step(s_)
+    stream.wait_stream(down)                    # every step's results are on the host
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e_steps, device)
     assert ws.status() == 0, "device status flags set during the e2e steps"
-    # the e2e results are the device results: the last step's outputs reached the host intact
-    for t, te, hdst in zip(L, L_e2e, host_out):
-        assert torch.equal(hdst.view(torch.int16), te["out"].cpu().view(torch.int16))
-        assert torch.equal(te["out"].view(torch.int16), t["out"].view(torch.int16))
+    # the e2e results are the device results: the outputs that reached the host are the step's
+    for si in range(nsets):
+        for t, te, hdst in zip(L, L_e2e[si], host_out[si]):
+            assert torch.equal(hdst.view(torch.int16), te["out"].cpu().view(torch.int16))
+            assert torch.equal(te["out"].view(torch.int16), t["out"].view(torch.int16))
 
     prefill = None
     if rank == 0 and not args.no_prefill:
@@ -594,7 +613,8 @@ def main():
         "e2e": {"value": job_throughput(tokens, e2e_ms, world), "unit": "new tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "mode": "one graph per layer; each layer's inputs in one pinned buffer (one upload per layer); "
-                        "uploads and downloads overlap the neighbouring layers' kernels on two copy streams"},
+                        "uploads and downloads overlap the neighbouring layers' kernels on two copy streams; "
+                        "two sets of device buffers, so a step's uploads overlap the previous step"},
         "gpu_launches": 3 * len(L),
         "clocks": clocks,
         "prefill": prefill,
