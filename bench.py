@@ -102,7 +102,9 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}_{os.getpid()}.csv")
+        import tempfile
+
+        self.path = os.path.join(tempfile.gettempdir(), f"hstu_bench_clocks_gpu{index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
@@ -130,6 +132,7 @@ class ClockSampler:
                     parts = [p.strip() for p in line.split(",")]
                     if len(parts) >= 9:
                         rows.append(parts)
+            os.remove(self.path)
         except OSError:
             pass
 

@@ -1,5 +1,5 @@
 // sm100.cuh -- thin inline-PTX wrappers for Blackwell (sm_100a): mbarriers, TMA tensor
-// loads (no multicast), tcgen05 tensor-memory allocation, MMA, commit and loads.
+// loads (each into its own CTA), tcgen05 tensor-memory allocation, MMA, commit and loads.
 #pragma once
 
 #include <cuda.h>
@@ -201,7 +201,7 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthread
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// ------------------------------------------------------------------ TMA (tiled, no multicast)
+// ------------------------------------------------------------------ TMA (tiled, one CTA per copy)
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* tm, uint32_t dst_smem, uint64_t* bar, int32_t c0,
                                             int32_t c1)
 {
