@@ -40,18 +40,24 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 # LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for the kernel
 # sources they were taken from (hash below); otherwise the bench reports traffic as null.
 PAGED_TRAFFIC_BYTES = 41.923328e6 + 3.84e3 + 6.571008e6
-PAGED_TRAFFIC_SOURCES = "9aba6c94d90c828c"
+PAGED_TRAFFIC_SOURCES = "fb7c6ce90c26ea98"
 # the same capture for the jagged prefill attention kernel (profiles/attn_tc_jagged_prefill_8users.md)
 PREFILL_TRAFFIC_BYTES = 63.268352e6 + 11.785728e6
 
 
 def kernel_sources_hash() -> str:
+    """Hash of the two kernels' source code with comments and blank space removed (editing a
+    comment does not change the kernel the counters were taken from)."""
     import hashlib
+    import re
 
     h = hashlib.sha256()
     for f in ("attn_tc.cu", "combine.cu"):
-        with open(os.path.join(ROOT, "hstu_attention_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "hstu_attention_b200", "csrc", f), encoding="utf-8") as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", " ", src).strip().encode())
     return h.hexdigest()[:16]
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 

@@ -31,6 +31,13 @@
 //               SiLU(x) = x/2 * (1 + tanh(x/2)), and store it as bf16 P into TMEM (P buffer
 //               t%2), where the P V MMA reads it.  The 1/n_max scale is applied to O once,
 //               when it leaves TMEM.
+//   epilogue    O / n_max leaves TMEM row per thread into a padded fp32 tile in the (then
+//               idle) K and V rings; each pointwise warp then stores whole 512-byte rows.
+// Grid: paged -- one CTA per piece of a balanced plan every CTA computes from the lengths
+// (plan_unit); jagged -- (head, user) x query block, heaviest query blocks first.  With
+// HSTU_FLAG_OVERLAP_PREVIOUS the grid is a programmatic dependent of the previous kernel: the
+// plan, page-id staging and set-up run early, and every access to inputs or the workspace waits
+// for that kernel (griddepcontrol.wait).
 // TMEM columns: S0 [0,128) | S1 [128,256) | O [256,384) | P0 [384,448) | P1 [448,512)
 // Shared memory (1024-byte aligned, 128B swizzle for every MMA operand):
 //   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 2 bias windows | bucket bounds | rab | page ids |

@@ -34,7 +34,8 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *     default stream).  They do not synchronise and allocate no device memory.
  *   - Scratch lives in a caller-provided workspace of at least hstu_workspace_size()
- *     bytes, 256-byte aligned, zeroed once with hstu_workspace_init() before first use.
+ *     bytes, 256-byte aligned, zeroed once with hstu_workspace_init() before first use
+ *     (hstu_attn_paged_fwd_noalloc uses a built-in scratch instead).
  *     One workspace must not be used by two calls that may run concurrently.
  *   - Host-detectable argument errors return a negative hstu_status_code and launch
  *     nothing.  Errors only the device can see (a page id out of range, lengths that do
