@@ -51,6 +51,9 @@ def bind(lib):
     lib.oracle_hstu_paged.restype = ctypes.c_int
     lib.oracle_hstu_paged.argtypes = [i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                       vp, vp, vp, vp, i32, vp, i32, i64, dbl, vp, i64, vp, vp, i32]
+    lib.oracle_hstu_jagged_bwd.restype = ctypes.c_int
+    lib.oracle_hstu_jagged_bwd.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i64,
+                                           ctypes.c_double, vp, vp, vp, vp, vp]
     lib.oracle_kv_append.restype = ctypes.c_int64
     lib.oracle_kv_append.argtypes = [i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp,
                                      vp, vp, vp]
@@ -128,6 +131,26 @@ def hstu_jagged(q, k, v, u, seq_offsets, num_targets, rab, n_max, eps=1e-5, rows
     if rc != 0:
         raise ValueError(f"oracle_hstu_jagged: inconsistent inputs (rc={rc})")
     return (out, o) if return_o else out
+
+
+def hstu_jagged_bwd(q, k, v, u, dout, seq_offsets, num_targets, rab, n_max, eps=1e-5):
+    """Gradients of the jagged prefill for upstream gradient ``dout`` (same shape and element
+    type as q).  Returns float64 (dq, dk, dv, du) [T, H, D] and drab [H, NB]."""
+    (q, k, v, u, dout), et = _same_type(q, k, v, u, dout)
+    T, H, D = q.shape
+    off = np.ascontiguousarray(seq_offsets, dtype=np.int64)
+    nt = np.ascontiguousarray(num_targets, dtype=np.int64)
+    B = off.shape[0] - 1
+    rab = np.ascontiguousarray(rab, dtype=np.float32)
+    assert rab.shape[0] == H
+    dq, dk, dv, du = (np.zeros((T, H, D), dtype=np.float64) for _ in range(4))
+    drab = np.zeros(rab.shape, dtype=np.float64)
+    rc = _load().oracle_hstu_jagged_bwd(B, H, D, _ptr(off), _ptr(nt), _ptr(q), _ptr(k), _ptr(v), _ptr(u),
+                                        _ptr(dout), et, _ptr(rab), rab.shape[1], int(n_max), float(eps),
+                                        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(du), _ptr(drab))
+    if rc != 0:
+        raise ValueError(f"oracle_hstu_jagged_bwd: inconsistent inputs (rc={rc})")
+    return dq, dk, dv, du, drab
 
 
 def hstu_paged(q_new, k_new, v_new, u_new, k_pages, v_pages, page_table, cached_lens, new_lens,

@@ -476,3 +476,125 @@ int64_t oracle_kv_append(int32_t B, int32_t H, int32_t D, int32_t page_size, int
     }
     return -bad;
 }
+
+/* ------------------------------------------------------------------ jagged backward */
+
+/*
+ * Gradients of the jagged forward above for a given upstream gradient dout = dL/d out
+ * (the backward pass of the same definition, by the chain rule, in float64):
+ *
+ *   out  = xhat * u,  xhat = (o - mean) * rstd      (per token, over its H*D vector)
+ *   du   = xhat * dout
+ *   dy   = dout * u
+ *   do   = rstd * (dy - mean(dy) - xhat * mean(dy * xhat))        (LayerNorm backward)
+ *   for every allowed pair (i, j) of a user and head h:
+ *     s    = q_i . k_j + rab[h][bucket(i - j)],  sig = sigmoid(s)
+ *     w    = s * sig / n_max
+ *     dw   = do_i . v_j
+ *     ds   = dw * sig * (1 + s * (1 - sig)) / n_max             (d SiLU(s) / ds)
+ *     dq_i += ds * k_j;  dk_j += ds * q_i;  dv_j += w * do_i;  drab[h][bucket(i - j)] += ds
+ *
+ * dq, dk, dv, du: [T][H][D] float64, drab: [H][NB] float64, all overwritten.  Pairs are taken
+ * in the order written (users, heads, queries, keys); no blocking or reordering.
+ * Returns 0, or -1 on inconsistent lengths.
+ */
+int oracle_hstu_jagged_bwd(int32_t B, int32_t H, int32_t D, const int64_t* seq_offsets,
+                           const int64_t* num_targets, const void* q, const void* k, const void* v,
+                           const void* u, const void* dout, int32_t elem_type, const float* rab,
+                           int32_t num_buckets, int64_t n_max, double eps, double* dq, double* dk,
+                           double* dv, double* du, double* drab)
+{
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t L = seq_offsets[b + 1] - seq_offsets[b];
+        if (L < 0 || num_targets[b] < 0 || num_targets[b] > L)
+            return -1;
+    }
+    const int64_t T = seq_offsets[B];
+    const int64_t HD = (int64_t)H * D;
+    const double inv_n = 1.0 / (double)n_max;
+    memset(dq, 0, sizeof(double) * (size_t)(T * HD));
+    memset(dk, 0, sizeof(double) * (size_t)(T * HD));
+    memset(dv, 0, sizeof(double) * (size_t)(T * HD));
+    memset(du, 0, sizeof(double) * (size_t)(T * HD));
+    memset(drab, 0, sizeof(double) * (size_t)((int64_t)H * num_buckets));
+    double* o = (double*)malloc(sizeof(double) * (size_t)(HD > 0 ? HD : 1));
+    double* dO = (double*)malloc(sizeof(double) * (size_t)(T * HD > 0 ? T * HD : 1));
+    for (int32_t b = 0; b < B; ++b) {
+        const int64_t s0 = seq_offsets[b], L = seq_offsets[b + 1] - s0;
+        const int64_t hist = L - num_targets[b];
+        /* forward o and the LayerNorm backward, token by token */
+        for (int64_t i = 0; i < L; ++i) {
+            for (int32_t h = 0; h < H; ++h)
+                for (int32_t c = 0; c < D; ++c) {
+                    double acc = 0.0;
+                    for (int64_t j = 0; j < L; ++j) {
+                        int allowed = (j <= i && j < hist) || (i >= hist && j == i);
+                        if (!allowed)
+                            continue;
+                        double s = 0.0;
+                        for (int32_t e = 0; e < D; ++e)
+                            s += ld(q, (s0 + i) * HD + (int64_t)h * D + e, elem_type) *
+                                 ld(k, (s0 + j) * HD + (int64_t)h * D + e, elem_type);
+                        s += (double)rab[(int64_t)h * num_buckets + oracle_bucket(i - j, n_max, num_buckets)];
+                        acc += s * sigmoid(s) * inv_n * ld(v, (s0 + j) * HD + (int64_t)h * D + c, elem_type);
+                    }
+                    o[(int64_t)h * D + c] = acc;
+                }
+            double mean = 0.0;
+            for (int64_t e = 0; e < HD; ++e)
+                mean += o[e];
+            mean /= (double)HD;
+            double var = 0.0;
+            for (int64_t e = 0; e < HD; ++e)
+                var += (o[e] - mean) * (o[e] - mean);
+            var /= (double)HD;
+            const double rstd = 1.0 / sqrt(var + eps);
+            double mdy = 0.0, mdyx = 0.0;
+            for (int64_t e = 0; e < HD; ++e) {
+                const int64_t idx = (s0 + i) * HD + e;
+                const double xhat = (o[e] - mean) * rstd;
+                const double g = ld(dout, idx, elem_type);
+                du[idx] = xhat * g;
+                const double dy = g * ld(u, idx, elem_type);
+                mdy += dy;
+                mdyx += dy * xhat;
+            }
+            mdy /= (double)HD;
+            mdyx /= (double)HD;
+            for (int64_t e = 0; e < HD; ++e) {
+                const int64_t idx = (s0 + i) * HD + e;
+                const double xhat = (o[e] - mean) * rstd;
+                const double dy = ld(dout, idx, elem_type) * ld(u, idx, elem_type);
+                dO[idx] = rstd * (dy - mdy - xhat * mdyx);
+            }
+        }
+        /* attention backward over the allowed pairs */
+        for (int32_t h = 0; h < H; ++h)
+            for (int64_t i = 0; i < L; ++i)
+                for (int64_t j = 0; j < L; ++j) {
+                    int allowed = (j <= i && j < hist) || (i >= hist && j == i);
+                    if (!allowed)
+                        continue;
+                    const int64_t qi = (s0 + i) * HD + (int64_t)h * D, kj = (s0 + j) * HD + (int64_t)h * D;
+                    const int bk = oracle_bucket(i - j, n_max, num_buckets);
+                    double s = 0.0, dw = 0.0;
+                    for (int32_t e = 0; e < D; ++e) {
+                        s += ld(q, qi + e, elem_type) * ld(k, kj + e, elem_type);
+                        dw += dO[qi + e] * ld(v, kj + e, elem_type);
+                    }
+                    s += (double)rab[(int64_t)h * num_buckets + bk];
+                    const double sig = sigmoid(s);
+                    const double w = s * sig * inv_n;
+                    const double ds = dw * sig * (1.0 + s * (1.0 - sig)) * inv_n;
+                    for (int32_t e = 0; e < D; ++e) {
+                        dq[qi + e] += ds * ld(k, kj + e, elem_type);
+                        dk[kj + e] += ds * ld(q, qi + e, elem_type);
+                        dv[kj + e] += w * dO[qi + e];
+                    }
+                    drab[(int64_t)h * num_buckets + bk] += ds;
+                }
+    }
+    free(o);
+    free(dO);
+    return 0;
+}

@@ -15,6 +15,7 @@ import tempfile
 import pytest
 
 import oracle
+from tests import test_oracle_bwd_pins as bwd_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "hstu_oracle.c")
@@ -42,6 +43,14 @@ MUTANTS = {
                                "int64_t idx = (((int64_t)page * P + j % P) * H + h) * D + c;"),
     "paged_query_position": ("int64_t i = C + (t - J->new_offsets[b]);", "int64_t i = t - J->new_offsets[b];"),
     "append_slot": ("int64_t slot = pos % page_size;", "int64_t slot = t % page_size;"),
+    # backward pass
+    "bwd_silu_derivative": ("const double ds = dw * sig * (1.0 + s * (1.0 - sig)) * inv_n;",
+                            "const double ds = dw * sig * inv_n;"),
+    "bwd_ln_mean_term": ("dO[idx] = rstd * (dy - mdy - xhat * mdyx);", "dO[idx] = rstd * (dy - xhat * mdyx);"),
+    "bwd_dv_weight": ("dv[kj + e] += w * dO[qi + e];", "dv[kj + e] += ds * dO[qi + e];"),
+    "bwd_dk_operand": ("dk[kj + e] += ds * ld(q, qi + e, elem_type);", "dk[kj + e] += ds * ld(k, qi + e, elem_type);"),
+    "bwd_drab_term": ("drab[(int64_t)h * num_buckets + bk] += ds;", "drab[(int64_t)h * num_buckets + bk] += dw;"),
+    "bwd_du_gate": ("du[idx] = xhat * g;", "du[idx] = g;"),
 }
 
 PIN_TESTS = [
@@ -55,6 +64,8 @@ PIN_TESTS = [
     pins.test_candidates_do_not_see_each_other,
     pins.test_append_scatter_and_roundtrip,
     pins.test_append_from_empty_then_paged_equals_jagged,
+    lambda: bwd_pins.test_gradients_match_finite_differences(3),
+    bwd_pins.test_zero_gate_blocks_attention_gradients,
 ]
 
 
