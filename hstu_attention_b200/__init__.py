@@ -42,6 +42,8 @@ EXPORTED = (
     "hstu_workspace_init",
     "hstu_read_status",
     "hstu_attn_jagged_fwd",
+    "hstu_attn_jagged_bwd",
+    "hstu_workspace_size_bwd",
     "hstu_attn_paged_fwd",
     "hstu_attn_paged_fwd_noalloc",
     "hstu_kv_append",
@@ -93,6 +95,11 @@ def load(path: Optional[str] = None):
             lib.hstu_read_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
             lib.hstu_attn_jagged_fwd.restype = ctypes.c_int
             lib.hstu_attn_jagged_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, sz, vp]
+            lib.hstu_workspace_size_bwd.restype = sz
+            lib.hstu_workspace_size_bwd.argtypes = [pp, i64]
+            lib.hstu_attn_jagged_bwd.restype = ctypes.c_int
+            lib.hstu_attn_jagged_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64,
+                                                 i32, vp, sz, vp]
             lib.hstu_attn_paged_fwd.restype = ctypes.c_int
             lib.hstu_attn_paged_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                 vp, sz, vp]
@@ -172,6 +179,40 @@ class Workspace:
         flags = ctypes.c_uint32(0)
         _check(load().hstu_read_status(self.ptr, _stream(stream), ctypes.byref(flags), int(clear)), "hstu_read_status")
         return int(flags.value)
+
+
+class BwdWorkspace(Workspace):
+    """Device scratch of the backward pass (status word + the recomputed o and its gradient)."""
+
+    def __init__(self, p: HstuParams, max_tokens: int, device=None, stream=None):
+        import torch
+
+        n = load().hstu_workspace_size_bwd(ctypes.byref(p), int(max_tokens))
+        if n == 0:
+            raise HstuError("hstu_workspace_size_bwd: invalid parameters")
+        self.nbytes = int(n)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        base = self.buf.data_ptr()
+        self.offset = (-base) % 256
+        self.ptr = base + self.offset
+        _check(load().hstu_workspace_init(self.ptr, self.nbytes, _stream(stream)), "hstu_workspace_init")
+
+
+def jagged_bwd(p: HstuParams, q, k, v, u, seq_offsets, num_targets, rab, dout, *, max_seqlen: int,
+               workspace: BwdWorkspace, stream=None):
+    """hstu_attn_jagged_bwd: gradients of sum(dout * out) of jagged_fwd.  Returns fp32
+    (dq, dk, dv, du) [T, H, D] and drab [H, NB]."""
+    import torch
+
+    dq, dk, dv, du = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(4))
+    drab = torch.empty(rab.shape, dtype=torch.float32, device=q.device)
+    B = seq_offsets.shape[0] - 1
+    rc = load().hstu_attn_jagged_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(seq_offsets),
+                                     _ptr(num_targets), _ptr(rab), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(du),
+                                     _ptr(drab), B, q.shape[0], int(max_seqlen), workspace.ptr, workspace.nbytes,
+                                     _stream(stream))
+    _check(rc, "hstu_attn_jagged_bwd")
+    return dq, dk, dv, du, drab
 
 
 def jagged_fwd(p: HstuParams, q, k, v, u, seq_offsets, num_targets, rab, *, max_seqlen: int, workspace: Workspace,

@@ -334,28 +334,12 @@ int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages,
     return finish(static_cast<cudaStream_t>(stream));
 }
 
-int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const void* k, const void* v, const void* u,
-                         const int32_t* seq_offsets, const int32_t* num_targets, const float* rab, void* out,
-                         int32_t B, int64_t total_tokens, int32_t max_seqlen, void* workspace,
-                         size_t workspace_bytes, void* stream)
+// The attention part of the jagged forward: O / n_max of every query row into the fp32 plane
+// `part` ([tokens][H][D]); device-detected errors go to the workspace status word.
+static int jagged_attention(const hstu_attn_params* params, const void* q, const void* k, const void* v,
+                            const int32_t* seq_offsets, const int32_t* num_targets, const float* rab, int32_t B,
+                            int64_t total_tokens, int32_t max_seqlen, void* workspace, float* part, cudaStream_t s)
 {
-    int rc = check_params(params, false);
-    if (rc != HSTU_OK)
-        return rc;
-    if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
-        return HSTU_ERR_INVALID_ARG;
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-        return HSTU_ERR_WORKSPACE;
-    if (B == 0 || total_tokens == 0 || max_seqlen == 0)
-        return HSTU_OK;
-    if (!q || !k || !v || !u || !out || !seq_offsets || !rab)
-        return HSTU_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out))
-        return HSTU_ERR_INVALID_ARG;
-    if (workspace_bytes < kStatusBytes + counts_bytes(total_tokens) + partial_bytes(params, 1, total_tokens))
-        return HSTU_ERR_WORKSPACE;
-    float* part = partials(workspace, total_tokens);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const double ln_nmax = log((double)params->n_max);
     const bool fp32 = params->dtype == HSTU_DTYPE_FP32;
     if (use_tc(params)) {
@@ -410,8 +394,102 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
         a.ln_nmax = ln_nmax;
         launch_attn_simt(a, false, fp32, B, s);
     }
+    return HSTU_OK;
+}
+
+int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const void* k, const void* v, const void* u,
+                         const int32_t* seq_offsets, const int32_t* num_targets, const float* rab, void* out,
+                         int32_t B, int64_t total_tokens, int32_t max_seqlen, void* workspace,
+                         size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, false);
+    if (rc != HSTU_OK)
+        return rc;
+    if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (B == 0 || total_tokens == 0 || max_seqlen == 0)
+        return HSTU_OK;
+    if (!q || !k || !v || !u || !out || !seq_offsets || !rab)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(out))
+        return HSTU_ERR_INVALID_ARG;
+    if (workspace_bytes < kStatusBytes + counts_bytes(total_tokens) + partial_bytes(params, 1, total_tokens))
+        return HSTU_ERR_WORKSPACE;
+    float* part = partials(workspace, total_tokens);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool fp32 = params->dtype == HSTU_DTYPE_FP32;
+    rc = jagged_attention(params, q, k, v, seq_offsets, num_targets, rab, B, total_tokens, max_seqlen, workspace, part,
+                          s);
+    if (rc != HSTU_OK)
+        return rc;
     launch_ln_gate(part, 1, nullptr, total_tokens, params->num_heads * params->head_dim, u, out, fp32, params->ln_eps,
                    s);
+    return finish(s);
+}
+
+size_t hstu_workspace_size_bwd(const hstu_attn_params* params, int64_t max_tokens)
+{
+    if (check_params(params, false) != HSTU_OK || max_tokens < 0)
+        return 0;
+    const size_t bytes = kStatusBytes + 2 * partial_bytes(params, 1, max_tokens);   // o, then d o
+    return (bytes + 255) & ~(size_t)255;
+}
+
+int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const void* k, const void* v, const void* u,
+                         const int32_t* seq_offsets, const int32_t* num_targets, const float* rab, const void* dout,
+                         float* dq, float* dk, float* dv, float* du, float* drab, int32_t B, int64_t total_tokens,
+                         int32_t max_seqlen, void* workspace, size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, false);
+    if (rc != HSTU_OK)
+        return rc;
+    if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (!drab)
+        return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // drab accumulates over pairs: it starts from zero (also for an empty batch)
+    if (cudaMemsetAsync(drab, 0, sizeof(float) * (size_t)params->num_heads * params->num_buckets, s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    if (B == 0 || total_tokens == 0 || max_seqlen == 0)
+        return finish(s);
+    if (!q || !k || !v || !u || !dout || !dq || !dk || !dv || !du || !seq_offsets || !rab)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(du))
+        return HSTU_ERR_INVALID_ARG;
+    if (workspace_bytes < kStatusBytes + 2 * partial_bytes(params, 1, total_tokens))
+        return HSTU_ERR_WORKSPACE;
+    float* o = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
+    const int64_t HD = (int64_t)params->num_heads * params->head_dim;
+    rc = jagged_attention(params, q, k, v, seq_offsets, num_targets, rab, B, total_tokens, max_seqlen, workspace, o, s);
+    if (rc != HSTU_OK)
+        return rc;
+    BwdArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.seq_offsets = seq_offsets;
+    a.num_targets = num_targets;
+    a.rab = rab;
+    a.dO = o + total_tokens * HD;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.drab = drab;
+    a.total_tokens = total_tokens;
+    a.B = B;
+    a.H = params->num_heads;
+    a.D = params->head_dim;
+    a.NB = params->num_buckets;
+    a.n_max = params->n_max;
+    a.ln_nmax = log((double)params->n_max);
+    a.inv_n = (float)(1.0 / (double)params->n_max);
+    launch_jagged_bwd(a, o, u, dout, du, params->ln_eps, params->dtype == HSTU_DTYPE_FP32, s);
     return finish(s);
 }
 

@@ -67,6 +67,24 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
 // counts == nullptr: every token has S partial planes; otherwise token t has counts[t].
 void launch_ln_gate(const float* part, int32_t S, const int32_t* counts, int64_t ntok, int32_t HD, const void* u,
                     void* out, bool fp32, float eps, cudaStream_t stream);
+// Backward pass of the jagged attention (attn_bwd.cu).
+struct BwdArgs {
+    const void *q, *k, *v;                 // [tokens][H][D], params dtype
+    const int32_t* seq_offsets;
+    const int32_t* num_targets;
+    const float* rab;                      // [H][NB]
+    float* dO;                             // [tokens][H][D] fp32: gradient of o (workspace)
+    float *dq, *dk, *dv;                   // [tokens][H][D] fp32, written
+    float* drab;                           // [H][NB] fp32, accumulated (zeroed by the caller)
+    int64_t total_tokens;
+    int32_t B, H, D, NB, n_max;
+    double ln_nmax;
+    float inv_n;
+};
+
+void launch_jagged_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du, float eps,
+                       bool fp32, cudaStream_t stream);
+
 void launch_attn_simt(const SimtArgs& a, bool paged, bool fp32, int32_t B, cudaStream_t stream);
 void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
                     cudaStream_t stream);

@@ -148,6 +148,35 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
                          size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace bytes for hstu_attn_jagged_bwd with at most max_tokens tokens: the status block and
+ * two fp32 [tokens][H][D] planes (the recomputed o and its gradient).  0 for invalid params.
+ */
+size_t hstu_workspace_size_bwd(const hstu_attn_params* params, int64_t max_tokens);
+
+/*
+ * Backward pass of hstu_attn_jagged_fwd: the gradients of sum(dout * out) with respect to the
+ * inputs, for the same arguments and an upstream gradient dout [total_tokens][H][D] (params
+ * dtype).  Outputs are fp32 and overwritten:
+ *   dq, dk, dv, du : [total_tokens][H][D]
+ *   drab           : [H][NB] (zeroed, then accumulated over every allowed pair)
+ * With o recomputed by the forward attention kernels, xhat = (o - mean) * rstd per token:
+ *   du = xhat * dout;  do = rstd * (dy - mean(dy) - xhat * mean(dy * xhat)),  dy = dout * u
+ *   per allowed pair (i, j), s = q_i . k_j + rab[h][bucket(i - j)], sig = sigmoid(s):
+ *   ds = (do_i . v_j) * sig * (1 + s * (1 - sig)) / n_max
+ *   dq_i += ds k_j,  dk_j += ds q_i,  dv_j += (s * sig / n_max) do_i,  drab[h][bucket] += ds
+ * The workspace must hold hstu_workspace_size_bwd(params, total_tokens) bytes (256-byte aligned,
+ * zeroed once with hstu_workspace_init); device-detected errors go to its status word as in the
+ * forward.  The pages train HSTU but print no backward pass; this is the chain rule applied to
+ * the forward definition above (sources as for hstu_attn_jagged_fwd).
+ */
+int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const void* k,
+                         const void* v, const void* u, const int32_t* seq_offsets,
+                         const int32_t* num_targets, const float* rab, const void* dout,
+                         float* dq, float* dk, float* dv, float* du, float* drab, int32_t B,
+                         int64_t total_tokens, int32_t max_seqlen, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
  * Paged cache hit: only the new tokens of each user are queries.  User b's keys are its
  * cached_lens[b] history tokens, read through page_table[b] (logical position p lives in
  * page page_table[b][p / P], slot p % P), followed by its new_lens[b] new tokens.  New
