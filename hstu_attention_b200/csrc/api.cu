@@ -451,19 +451,23 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
         return HSTU_ERR_WORKSPACE;
     if (!drab)
         return HSTU_ERR_INVALID_ARG;
+    const bool empty = B == 0 || total_tokens == 0 || max_seqlen == 0;
+    if (!empty) {
+        // every host-detectable error is reported before anything is enqueued
+        if (!q || !k || !v || !u || !dout || !dq || !dk || !dv || !du || !seq_offsets || !rab)
+            return HSTU_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(dout) || !aligned16(dq) ||
+            !aligned16(dk) || !aligned16(dv) || !aligned16(du))
+            return HSTU_ERR_INVALID_ARG;
+        if (workspace_bytes < kStatusBytes + 2 * partial_bytes(params, 1, total_tokens))
+            return HSTU_ERR_WORKSPACE;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // drab accumulates over pairs: it starts from zero (also for an empty batch)
     if (cudaMemsetAsync(drab, 0, sizeof(float) * (size_t)params->num_heads * params->num_buckets, s) != cudaSuccess)
         return HSTU_ERR_CUDA;
-    if (B == 0 || total_tokens == 0 || max_seqlen == 0)
+    if (empty)
         return finish(s);
-    if (!q || !k || !v || !u || !dout || !dq || !dk || !dv || !du || !seq_offsets || !rab)
-        return HSTU_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(dout) || !aligned16(dq) ||
-        !aligned16(dk) || !aligned16(dv) || !aligned16(du))
-        return HSTU_ERR_INVALID_ARG;
-    if (workspace_bytes < kStatusBytes + 2 * partial_bytes(params, 1, total_tokens))
-        return HSTU_ERR_WORKSPACE;
     float* o = reinterpret_cast<float*>(static_cast<char*>(workspace) + kStatusBytes);
     const int64_t HD = (int64_t)params->num_heads * params->head_dim;
     rc = jagged_attention(params, q, k, v, seq_offsets, num_targets, rab, B, total_tokens, max_seqlen, workspace, o, s);

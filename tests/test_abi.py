@@ -119,3 +119,32 @@ def test_flags_and_noalloc_limit_without_gpu(lib):
     misaligned_flags = list(args)
     misaligned_flags[-2] = fake + 2                                       # flags_out not 4-byte aligned
     assert N(ctypes.byref(_p(n_max=8192)), *misaligned_flags) == -1
+
+
+def test_backward_host_validation_without_gpu(lib):
+    """The backward entry rejects bad arguments before it enqueues anything."""
+    p = _p()
+    fake = 1 << 20
+    ws = 1 << 24
+    n = lib.hstu_workspace_size_bwd(ctypes.byref(p), 1000)
+    assert n % 256 == 0 and n >= 256 + 2 * 1000 * 4 * 128 * 4
+    assert lib.hstu_workspace_size_bwd(None, 10) == 0
+    Bw = lib.hstu_attn_jagged_bwd
+    args = [fake] * 4 + [fake, None, fake, fake] + [fake] * 5 + [2, 100, 64, ws, 1 << 30, None]
+    assert Bw(None, *args) == -1
+    assert Bw(ctypes.byref(_p(head_dim=96)), *args) == -2
+    no_drab = list(args)
+    no_drab[12] = None
+    assert Bw(ctypes.byref(p), *no_drab) == -1
+    no_dout = list(args)
+    no_dout[7] = None
+    assert Bw(ctypes.byref(p), *no_dout) == -1
+    mis = list(args)
+    mis[8] = fake + 4                                                     # dq not 16-byte aligned
+    assert Bw(ctypes.byref(p), *mis) == -1
+    small = list(args)
+    small[-2] = 1000                                                      # workspace too small
+    assert Bw(ctypes.byref(p), *small) == -3
+    unal = list(args)
+    unal[-3] = ws + 8
+    assert Bw(ctypes.byref(p), *unal) == -3
