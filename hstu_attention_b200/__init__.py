@@ -148,6 +148,27 @@ def _ptr(t) -> Optional[int]:
     return t.data_ptr()
 
 
+def _check_args(p: HstuParams, elems=(), ints=(), floats=()):
+    """Element types and shapes the C ABI expects (it receives bare pointers and cannot tell):
+    token tensors [T, H, D] and pages of the params dtype, index arrays int32, rab fp32."""
+    import torch
+
+    want = torch.bfloat16 if p.dtype == HSTU_DTYPE_BF16 else torch.float32
+    for name, t in elems:
+        if t is None:
+            continue
+        if t.dtype != want:
+            raise HstuError(f"{name} must be {want}, got {t.dtype}")
+        if t.dim() < 3 or t.shape[-1] != p.head_dim or (t.dim() == 3 and t.shape[1] != p.num_heads):
+            raise HstuError(f"{name} has shape {tuple(t.shape)}; expected [..., H={p.num_heads}, D={p.head_dim}]")
+    for name, t in ints:
+        if t is not None and t.dtype != torch.int32:
+            raise HstuError(f"{name} must be int32, got {t.dtype}")
+    for name, t in floats:
+        if t is not None and t.dtype != torch.float32:
+            raise HstuError(f"{name} must be float32, got {t.dtype}")
+
+
 def _stream(stream) -> int:
     import torch
 
@@ -204,6 +225,8 @@ def jagged_bwd(p: HstuParams, q, k, v, u, seq_offsets, num_targets, rab, dout, *
     (dq, dk, dv, du) [T, H, D] and drab [H, NB]."""
     import torch
 
+    _check_args(p, elems=(("q", q), ("k", k), ("v", v), ("u", u), ("dout", dout)),
+                ints=(("seq_offsets", seq_offsets), ("num_targets", num_targets)), floats=(("rab", rab),))
     dq, dk, dv, du = (torch.empty(q.shape, dtype=torch.float32, device=q.device) for _ in range(4))
     drab = torch.empty(rab.shape, dtype=torch.float32, device=q.device)
     B = seq_offsets.shape[0] - 1
@@ -221,6 +244,8 @@ def jagged_fwd(p: HstuParams, q, k, v, u, seq_offsets, num_targets, rab, *, max_
     rab [H, NB] fp32.  Returns out [T, H, D]."""
     import torch
 
+    _check_args(p, elems=(("q", q), ("k", k), ("v", v), ("u", u), ("out", out)),
+                ints=(("seq_offsets", seq_offsets), ("num_targets", num_targets)), floats=(("rab", rab),))
     if out is None:
         out = torch.empty_like(q)
     B = seq_offsets.shape[0] - 1
@@ -237,6 +262,10 @@ def paged_fwd(p: HstuParams, q_new, k_new, v_new, u_new, k_pages, v_pages, page_
     page_table [B, max_pages] int32; cached_lens/new_lens/num_targets [B] int32."""
     import torch
 
+    _check_args(p, elems=(("q_new", q_new), ("k_new", k_new), ("v_new", v_new), ("u_new", u_new),
+                          ("k_pages", k_pages), ("v_pages", v_pages), ("out", out)),
+                ints=(("page_table", page_table), ("cached_lens", cached_lens), ("new_lens", new_lens),
+                      ("num_targets", num_targets)), floats=(("rab", rab),))
     if out is None:
         out = torch.empty_like(q_new)
     B = cached_lens.shape[0]
@@ -255,6 +284,10 @@ def paged_fwd_noalloc(p: HstuParams, q_new, k_new, v_new, u_new, k_pages, v_page
     status bits.  All calls on a device share the scratch: do not overlap them across streams."""
     import torch
 
+    _check_args(p, elems=(("q_new", q_new), ("k_new", k_new), ("v_new", v_new), ("u_new", u_new),
+                          ("k_pages", k_pages), ("v_pages", v_pages), ("out", out)),
+                ints=(("page_table", page_table), ("cached_lens", cached_lens), ("new_lens", new_lens),
+                      ("num_targets", num_targets), ("flags", flags)), floats=(("rab", rab),))
     if out is None:
         out = torch.empty_like(q_new)
     B = cached_lens.shape[0]
@@ -269,6 +302,9 @@ def paged_fwd_noalloc(p: HstuParams, q_new, k_new, v_new, u_new, k_pages, v_page
 def kv_append(p: HstuParams, k_pages, v_pages, page_table, k_new, v_new, cached_lens, new_lens, num_targets, *,
               max_new: int, workspace: Workspace, stream=None):
     """hstu_kv_append: copy the first new_lens[b] - num_targets[b] new rows of each user into its pages."""
+    _check_args(p, elems=(("k_pages", k_pages), ("v_pages", v_pages), ("k_new", k_new), ("v_new", v_new)),
+                ints=(("page_table", page_table), ("cached_lens", cached_lens), ("new_lens", new_lens),
+                      ("num_targets", num_targets)))
     B = cached_lens.shape[0]
     rc = load().hstu_kv_append(ctypes.byref(p), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(k_new),
                                _ptr(v_new), _ptr(cached_lens), _ptr(new_lens), _ptr(num_targets), B,

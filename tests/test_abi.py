@@ -148,3 +148,24 @@ def test_backward_host_validation_without_gpu(lib):
     unal = list(args)
     unal[-3] = ws + 8
     assert Bw(ctypes.byref(p), *unal) == -3
+
+
+def test_binding_checks_types_before_any_call():
+    """The binding refuses tensors of the wrong element type or shape (the C ABI takes bare
+    pointers) before it touches the library or the device."""
+    import torch
+
+    p = hb.params(4, 128, torch.bfloat16, 16, 64)
+    t = torch.zeros((8, 4, 128), dtype=torch.bfloat16)
+    off = torch.tensor([0, 8], dtype=torch.int32)
+    rab = torch.zeros((4, 16))
+    with pytest.raises(hb.HstuError, match="q must be torch.bfloat16"):
+        hb.jagged_fwd(p, t.float(), t, t, t, off, None, rab, max_seqlen=8, workspace=None)
+    with pytest.raises(hb.HstuError, match="seq_offsets must be int32"):
+        hb.jagged_fwd(p, t, t, t, t, off.long(), None, rab, max_seqlen=8, workspace=None)
+    with pytest.raises(hb.HstuError, match="rab must be float32"):
+        hb.jagged_fwd(p, t, t, t, t, off, None, rab.double(), max_seqlen=8, workspace=None)
+    with pytest.raises(hb.HstuError, match="expected"):
+        hb.jagged_fwd(p, t[:, :2], t, t, t, off, None, rab, max_seqlen=8, workspace=None)
+    with pytest.raises(hb.HstuError, match="dout must be torch.bfloat16"):
+        hb.jagged_bwd(p, t, t, t, t, off, None, rab, t.float(), max_seqlen=8, workspace=None)
