@@ -12,7 +12,7 @@ deployment blog (KuaiRand-1K itself is not available here).
 Prints one JSON line (rank 0).  Under torchrun each rank runs its own replica of the batch
 on its own GPU (weak scaling, no collective on the data path); the time is the max over
 ranks.  The step is captured in one CUDA graph and timed with CUDA events; the 8 layers
-read ~370 MB of distinct pages per step, more than the 126 MB L2, so no flush is needed.
+read ~340 MB of distinct pages and tokens per step, more than the 126 MB L2, so no flush is needed.
 """
 from __future__ import annotations
 
@@ -606,7 +606,7 @@ def main():
                                "paged attention",
                    "global_batch": layers_cfg["B"] * world, "seq_len": int(max(int(c.cached_lens.max()) for c in layers)),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (8 layers of distinct pages, ~370 MB per step)",
+                   "l2": "inputs larger than L2 (8 layers of distinct pages, ~343 MB per step)",
                    "graph": "one CUDA graph per step; appends on a forked stream (they do not feed "
                             "the attention, which reads new keys from k_new)"},
         "roofline": {"bound": "hbm", "kernel": "hstu_attn_paged_fwd (attention kernel + LayerNorm-gate kernel)",
