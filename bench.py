@@ -35,13 +35,12 @@ from hstu_attention_b200 import inputs as gen  # noqa: E402
 METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline"
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per paged call on one layer of this
-# batch, from one `ncu --set full` capture (profiles/attn_tc_paged_cachehit_layer0.md):
-# attn_tc_kernel 41.923 MB + 3.8 KB, ln_gate_kernel 6.571 MB (ncu flushes caches, so the
-# LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for the kernel
-# sources they were taken from (hash below); otherwise the bench reports traffic as null.
+# batch, from one `ncu --set full` capture of the attention and LayerNorm kernels (ncu flushes
+# caches, so the LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for
+# the kernel sources they were taken from (hash below); otherwise the bench reports traffic as null.
 PAGED_TRAFFIC_BYTES = 41.923328e6 + 3.84e3 + 6.571008e6
 PAGED_TRAFFIC_SOURCES = "fb7c6ce90c26ea98"
-# the same capture for the jagged prefill attention kernel (profiles/attn_tc_jagged_prefill_8users.md)
+# the same kind of capture for the jagged prefill attention kernel
 PREFILL_TRAFFIC_BYTES = 63.268352e6 + 11.785728e6
 
 
@@ -52,7 +51,7 @@ def kernel_sources_hash() -> str:
     import re
 
     h = hashlib.sha256()
-    for f in ("attn_tc.cu", "combine.cu"):
+    for f in ("attn_tc.cu", "attn_paged.cu", "combine.cu"):
         with open(os.path.join(ROOT, "hstu_attention_b200", "csrc", f), encoding="utf-8") as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)

@@ -29,7 +29,6 @@ DEV_BAD_PAGE = 1 << 0
 DEV_BAD_LENGTH = 1 << 1
 DEV_BAD_NMAX = 1 << 2
 DEV_TIMEOUT = 1 << 3
-DEV_SMEM_ALIGN = 1 << 4
 
 ERR_SCRATCH_LIMIT = -5
 

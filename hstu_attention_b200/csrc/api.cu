@@ -373,7 +373,7 @@ static int jagged_attention(const hstu_attn_params* params, const void* q, const
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.timeout_ns = kTimeoutNs;
         a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
-        launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), false, B, s);
+        launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), B, s);
     } else {
         SimtArgs a{};
         a.q = q;
@@ -491,6 +491,7 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
     a.D = params->head_dim;
     a.NB = params->num_buckets;
     a.n_max = params->n_max;
+    a.max_seqlen = max_seqlen;
     a.ln_nmax = log((double)params->n_max);
     a.inv_n = (float)(1.0 / (double)params->n_max);
     launch_jagged_bwd(a, o, u, dout, du, params->ln_eps, params->dtype == HSTU_DTYPE_FP32, s);
@@ -518,6 +519,8 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
     if (!aligned16(q_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(u_new) || !aligned16(k_pages) ||
         !aligned16(v_pages) || !aligned16(out))
         return HSTU_ERR_INVALID_ARG;
+    if (use_tc(params) && B > paged_max_users())
+        return HSTU_ERR_UNSUPPORTED;
     const size_t one = partial_bytes(params, 1, total_new);
     const size_t fixed = kStatusBytes + counts_bytes(total_new);
     if (workspace_bytes < fixed + one)
@@ -566,7 +569,7 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.timeout_ns = kTimeoutNs;
         a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
-        launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), true, B, s);
+        launch_attn_paged(m, a, host_bounds(params->n_max, params->num_buckets), num_sms(), s);
     } else {
         SimtArgs a{};
         a.q = q_new;

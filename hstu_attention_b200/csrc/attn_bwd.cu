@@ -113,7 +113,9 @@ attn_bwd_dq_kernel(BwdArgs a)
     if (b >= 0) {
         const int64_t s0 = a.seq_offsets[b], L = a.seq_offsets[b + 1] - s0;
         const int32_t nt = a.num_targets ? a.num_targets[b] : 0;
-        const bool ok = s0 >= 0 && L > 0 && s0 + L <= a.total_tokens && nt >= 0 && nt <= L && L <= a.n_max;
+        // the forward's rule (jagged_geom): a rejected user has o = 0 and contributes nothing
+        const bool ok = s0 >= 0 && L > 0 && s0 + L <= a.total_tokens && nt >= 0 && nt <= L && L <= a.n_max &&
+                        L <= a.max_seqlen;
         const int64_t hist = L - nt, i = t - s0;
         const T* q = static_cast<const T*>(a.q);
         const T* k = static_cast<const T*>(a.k);
@@ -173,7 +175,9 @@ attn_bwd_dkv_kernel(BwdArgs a)
     if (b >= 0) {
         const int64_t s0 = a.seq_offsets[b], L = a.seq_offsets[b + 1] - s0;
         const int32_t nt = a.num_targets ? a.num_targets[b] : 0;
-        const bool ok = s0 >= 0 && L > 0 && s0 + L <= a.total_tokens && nt >= 0 && nt <= L && L <= a.n_max;
+        // the forward's rule (jagged_geom): a rejected user has o = 0 and contributes nothing
+        const bool ok = s0 >= 0 && L > 0 && s0 + L <= a.total_tokens && nt >= 0 && nt <= L && L <= a.n_max &&
+                        L <= a.max_seqlen;
         const int64_t hist = L - nt, j = t - s0;
         const T* q = static_cast<const T*>(a.q);
         const T* k = static_cast<const T*>(a.k);

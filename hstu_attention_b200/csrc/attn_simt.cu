@@ -36,14 +36,24 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtArgs a)
     const int64_t HD = (int64_t)H * D;
     if (threadIdx.x < 32) {
         UserGeom g = kPaged ? paged_geom(a.cached_lens, a.new_lens, a.num_targets, b, a.total_tokens, a.max_len,
-                                         a.max_pages * a.P, a.n_max, a.ws, qb == 0 && h == 0)
-                            : jagged_geom(a.seq_offsets, a.num_targets, b, a.total_tokens, a.max_len, a.n_max,
-                                          a.ws, qb == 0 && h == 0);
+                                         a.max_pages * a.P, a.n_max)
+                            : jagged_geom(a.seq_offsets, a.num_targets, b, a.total_tokens, a.max_len, a.n_max);
         if (threadIdx.x == 0)
             sG = g;
     }
     __syncthreads();
     const UserGeom g = sG;
+    if (!g.ok) {
+        // a rejected user: the q-block-0 CTA of each head zeroes that head's slice of every row
+        // of the user, including rows past the grid (a user longer than the host's bound)
+        if (qb == 0) {
+            if (h == 0 && threadIdx.x == 0)
+                set_flag(a.ws, g.flags);
+            for (int64_t x = threadIdx.x; x < (int64_t)g.N * D; x += kSimtThreads)
+                a.part[(g.tok0 + x / D) * HD + (int64_t)h * D + x % D] = 0.f;
+        }
+        return;
+    }
     const int r = threadIdx.x >> 2;            // query row within the block
     const int part = threadIdx.x & 3;          // channel quarter
     const int dq = D >> 2;                     // channels per thread

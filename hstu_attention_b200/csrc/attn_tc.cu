@@ -1,4 +1,5 @@
-// attn_tc.cu -- HSTU attention on Blackwell tensor cores (bf16 in, fp32 accumulate, D = 128).
+// attn_tc.cu -- jagged-prefill HSTU attention on Blackwell tensor cores (bf16 in, fp32
+// accumulate, D = 128).  (The paged cache hit has its own kernel, attn_paged.cu.)
 //
 // What it computes (per user b, head h): for a block of 128 query rows and the key tiles the
 // block may see,
@@ -8,16 +9,11 @@
 //     O / n_max -> workspace (fp32)
 // SiLU weighting replaces softmax, so there is no running max or row sum and key tiles can be
 // split across CTAs and summed afterwards (aitrends.kr summary, section "HSTU의 순차 모델링";
-// news.bpdata.com, section "HSTU").  Keys of the paged layout come from the per-user page
-// table for positions below cached_len and from the new-token rows after that (NVIDIA blog
-// "Deploying an HSTU Generative Recommender with NVIDIA Dynamo-Triton", section "Why serving
-// large sequential recommenders is hard": the attention kernel reads K/V from the paged
-// cache).  combine.cu applies LayerNorm(O) * U to the fp32 partial outputs.
+// news.bpdata.com, section "HSTU").  combine.cu applies LayerNorm(O) * U to the fp32 outputs.
 //
 // CTA roles (384 threads):
 //   warp 0      TMA producer of Q and of the K tiles (2-stage ring; a K stage frees as soon as
-//               Q K^T has read it).  Paged tiles are gathered page by page (one TMA box of P
-//               rows per page and channel half) using page ids staged in shared memory.
+//               Q K^T has read it).
 //   warp 3      TMA producer of the V tiles (3-stage ring, freed after P V).
 //   warp 1      allocates all 512 TMEM columns; lane 0 issues every MMA:
 //               S_t = Q K_t^T into S buffer t%2, then O += P_{t-1} V_{t-1}, so the pointwise
@@ -33,15 +29,13 @@
 //               when it leaves TMEM.
 //   epilogue    O / n_max leaves TMEM row per thread into a padded fp32 tile in the (then
 //               idle) K and V rings; each pointwise warp then stores whole 512-byte rows.
-// Grid: paged -- one CTA per piece of a balanced plan every CTA computes from the lengths
-// (plan_unit); jagged -- (head, user) x query block, heaviest query blocks first.  With
+// Grid: (head, user) x query block, heaviest query blocks first.  With
 // HSTU_FLAG_OVERLAP_PREVIOUS the grid is a programmatic dependent of the previous kernel: the
-// plan, page-id staging and set-up run early, and every access to inputs or the workspace waits
-// for that kernel (griddepcontrol.wait).
+// set-up runs early, and every access to inputs or the workspace -- the status word included --
+// waits for that kernel (griddepcontrol.wait).
 // TMEM columns: S0 [0,128) | S1 [128,256) | O [256,384) | P0 [384,448) | P1 [448,512)
 // Shared memory (1024-byte aligned, 128B swizzle for every MMA operand):
-//   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 2 bias windows | bucket bounds | rab | page ids |
-//   mbarriers
+//   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 2 bias windows | bucket bounds | rab | mbarriers
 // Every wait is bounded (HSTU_DEV_TIMEOUT) so a logic error cannot hang the GPU.
 #include <atomic>
 
@@ -58,7 +52,6 @@ constexpr int kKStages = 2;
 constexpr int kVStages = 3;
 constexpr int kTcThreads = 384;
 constexpr int kMaxNB = 1024;                  // buckets staged in shared memory
-constexpr int kMaxPageIds = 1024;             // page ids staged per CTA (rest read from global)
 constexpr uint32_t kHalf = 128 * 128;         // 128 rows x 128 bytes = 16 KB (one swizzle column)
 constexpr uint32_t kTileBytes = 2 * kHalf;    // one 128 x 128 bf16 operand
 constexpr uint32_t kOffQ = 0;
@@ -70,8 +63,7 @@ constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
 constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
-constexpr uint32_t kOffPages = kOffRab + kMaxNB * 4;
-constexpr uint32_t kOffBar = kOffPages + kMaxPageIds * 4;
+constexpr uint32_t kOffBar = kOffRab + kMaxNB * 4;
 constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1 + 2 + 2;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
@@ -85,23 +77,15 @@ static_assert(kOffK + kTile * kOStride * 4 <= kOffWin, "epilogue staging fits th
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 
 struct TileGeo {
-    int32_t j0;       // absolute position of key row 0 of the tile
+    int32_t j0;       // position of key row 0 of the tile
     int32_t kvend;    // keys at positions >= kvend are not valid data for this tile
-    bool cached;      // keys come from pages
 };
 
-__device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t ct, int32_t C, int32_t L)
+__device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t L)
 {
     TileGeo g;
-    if (t < ct) {
-        g.j0 = t * kTile;
-        g.kvend = C;
-        g.cached = true;
-    } else {
-        g.j0 = C + (t - ct) * kTile;
-        g.kvend = L;
-        g.cached = false;
-    }
+    g.j0 = t * kTile;
+    g.kvend = L;
     return g;
 }
 
@@ -181,230 +165,54 @@ __device__ int bucket_bound(int k, double ln_nmax, int nb)
     return c > 0x7ffffffe ? 0x7ffffffe : (int)c;
 }
 
-// ------------------------------------------------------------------ paged work plan
-// Entry e = user * qblocks + q-block.  Key tiles of an entry: the cached tiles plus the new-key
-// tiles up to the block's last query (qblk + 1 of them).  A user with invalid lengths keeps
-// one tile on q-block 0 so that one CTA writes its (zero) rows and flags it.
-__device__ __forceinline__ int entry_tiles(const TcArgs& a, int e)
-{
-    const int b = e / a.qblocks, q = e % a.qblocks;
-    const int32_t C = a.cached_lens[b], N = a.new_lens[b];
-    const int32_t T = a.num_targets ? a.num_targets[b] : 0;
-    const bool ok = C >= 0 && N >= 0 && T >= 0 && T <= N && N <= a.max_len && C <= a.max_pages * a.P;
-    if (!ok)
-        return q == 0 ? 1 : 0;
-    if (q * kTile >= N)
-        return 0;
-    return (C + kTile - 1) / kTile + q + 1;
-}
-
-// The entries' tile counts of this lane (entries lane, lane + 32, ...), read once.  Entries
-// past kPlanRounds * 32 are re-read when needed (the arrays are then in L1).
-constexpr int kPlanRounds = 8;
-struct PlanTiles {
-    int t[kPlanRounds];
-};
-
-// min(ceil(t / c), max_splits) for t >= 0, by comparisons (no integer division).
-__device__ __forceinline__ int splits_for(int t, int c, int max_splits)
-{
-    int s = 0;
-#pragma unroll
-    for (int k = 0; k < kMaxSplits; ++k)
-        s += ((k < max_splits) & (t > k * c)) ? 1 : 0;
-    return s;
-}
-
-// Tiles per piece c: start from ceil(all tiles over all heads / target_ctas) and grow until
-// the pieces fit the grid that was launched (gridDim.x >= H * entries bounds the count at
-// c = max tiles, so a fit always exists).  Whole warp.
-__device__ int plan_tiles_per_piece(const TcArgs& a, const PlanTiles& pt)
-{
-    const int lane = threadIdx.x & 31;
-    const int entries = a.B * a.qblocks;
-    int64_t w = 0;
-#pragma unroll
-    for (int r = 0; r < kPlanRounds; ++r)
-        w += pt.t[r];                                    // zero past the last entry
-    for (int e = lane + 32 * kPlanRounds; e < entries; e += 32)
-        w += entry_tiles(a, e);
-    for (int o = 16; o > 0; o >>= 1)
-        w += __shfl_xor_sync(0xffffffffu, w, o);
-    w *= a.H;
-    const int64_t tgt = a.target_ctas > 0 ? a.target_ctas : 1;
-    int c = (int)((w + tgt - 1) / tgt);
-    if (c < 1)
-        c = 1;
-    for (int it = 0; it < 64; ++it) {
-        int64_t units = 0;
-#pragma unroll
-        for (int r = 0; r < kPlanRounds; ++r)
-            units += splits_for(pt.t[r], c, a.max_splits);
-        for (int e = lane + 32 * kPlanRounds; e < entries; e += 32)
-            units += splits_for(entry_tiles(a, e), c, a.max_splits);
-        for (int o = 16; o > 0; o >>= 1)
-            units += __shfl_xor_sync(0xffffffffu, units, o);
-        if (units * a.H <= (int64_t)gridDim.x)
-            return c;
-        c += (c + 7) / 8;                     // grow by ~12% per step
-    }
-    return 0x3fffffff;                        // one piece per entry always fits the grid
-}
-
-// The piece this CTA (blockIdx.x) works on: entry e_out, index local_out within the entry and
-// the entry's number of splits (pieces are numbered entry by entry, H * splits(e) per entry).
-// Returns false past the last piece.  Whole warp.
-__device__ bool plan_unit(const TcArgs& a, int& e_out, int& local_out, int& nsplit_out)
-{
-    const int lane = threadIdx.x & 31;
-    const int entries = a.B * a.qblocks;
-    PlanTiles pt;
-#pragma unroll
-    for (int r = 0; r < kPlanRounds; ++r) {
-        const int e = lane + 32 * r;
-        pt.t[r] = e < entries ? entry_tiles(a, e) : 0;
-    }
-    const int c = plan_tiles_per_piece(a, pt);
-    const int want = (int)blockIdx.x;
-    int base = 0;
-    for (int r0 = 0, r = 0; r0 < entries; r0 += 32, ++r) {
-        const int e = r0 + lane;
-        int t = 0;
-#pragma unroll
-        for (int k = 0; k < kPlanRounds; ++k)
-            t = (k == r) ? pt.t[k] : t;                  // register select, no local memory
-        if (r >= kPlanRounds && e < entries)
-            t = entry_tiles(a, e);
-        const int ns = e < entries ? splits_for(t, c, a.max_splits) : 0;
-        const int units = a.H * ns;
-        int incl = units;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o)
-                incl += y;
-        }
-        const int excl = incl - units;
-        const bool mine = units > 0 && want >= base + excl && want < base + incl;
-        const unsigned who = __ballot_sync(0xffffffffu, mine);
-        if (who) {
-            const int src = __ffs(who) - 1;
-            e_out = __shfl_sync(0xffffffffu, e, src);
-            local_out = __shfl_sync(0xffffffffu, want - base - excl, src);
-            nsplit_out = __shfl_sync(0xffffffffu, ns, src);
-            return true;
-        }
-        base += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    return false;
-}
-
-template <bool kPaged>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
-               const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ BucketBounds bb,
-               const TcArgs a)
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ BucketBounds bb, const TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ UserGeom sG;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ int sUnit[5];
-    int b, qblk, h, split, nsplit;
-    if (kPaged) {
-        // balanced work plan: every (user, query block) entry's key tiles are cut into
-        // ceil(tiles / c) contiguous pieces, c chosen so that about target_ctas pieces exist
-        // over all heads; this CTA takes piece blockIdx.x (computed the same way by every CTA)
-        if (warp == 0) {
-            int e = -1, local = 0, ns = 1;
-            const bool found = plan_unit(a, e, local, ns);
-            if (lane == 0) {
-                sUnit[0] = found ? e : -1;                     // entry: user * qblocks + q-block
-                sUnit[1] = local;                              // piece index within the entry
-                sUnit[2] = found ? ns : 1;
-            }
-        }
-        __syncthreads();
-        if (sUnit[0] < 0) {
-            pdl_launch_dependents();
-            return;                                  // more CTAs than pieces
-        }
-        const int e = sUnit[0], local = sUnit[1];
-        b = e / a.qblocks;
-        qblk = e % a.qblocks;
-        nsplit = sUnit[2];
-        h = local / nsplit;
-        split = local % nsplit;
-    } else {
-        // grid: x = (head, user), y = query block, heaviest blocks first
-        h = blockIdx.x % a.H;
-        b = blockIdx.x / a.H;
-        qblk = a.qblocks - 1 - (int)blockIdx.y;
-        split = 0;
-        nsplit = 1;
-    }
-
-    extern __shared__ __align__(1024) uint8_t smem_pre[];
-    if (kPaged && (warp == 2 || warp == 3)) {
-        // the user's page-table row, loaded while warp 0 reads the lengths (page ids past the
-        // user's cached length are never used; invalid ids are caught when a page is used)
-        const uint32_t pre_pad = (1024u - (sm100::smem_u32(smem_pre) & 1023u)) & 1023u;
-        int32_t* rowbuf = reinterpret_cast<int32_t*>(smem_pre + pre_pad + kOffPages);
-        const int nrow = min(a.max_pages, kMaxPageIds);
-        for (int k = threadIdx.x - 64; k < nrow; k += 64)
-            rowbuf[k] = a.page_table[(int64_t)b * a.max_pages + k];
-    }
+    // grid: x = (head, user), y = query block, heaviest blocks first
+    const int h = blockIdx.x % a.H;
+    const int b = blockIdx.x / a.H;
+    const int qblk = a.qblocks - 1 - (int)blockIdx.y;
     if (warp == 0) {
-        const bool report = qblk == 0 && h == 0 && split == 0;
-        UserGeom g = kPaged ? paged_geom(a.cached_lens, a.new_lens, a.num_targets, b, a.total_tokens, a.max_len,
-                                         a.max_pages * a.P, a.n_max, a.ws, report)
-                            : jagged_geom(a.seq_offsets, a.num_targets, b, a.total_tokens, a.max_len, a.n_max,
-                                          a.ws, report);
+        UserGeom g = jagged_geom(a.seq_offsets, a.num_targets, b, a.total_tokens, a.max_len, a.n_max);
         if (lane == 0)
             sG = g;
     }
     __syncthreads();
     const UserGeom g = sG;
     const int32_t qrow0 = qblk * kTile;
+    const int64_t HD = (int64_t)a.H * kTcD;
+    float* part = a.part;
+    if (!g.ok) {
+        // a rejected user: the q-block-0 CTA of each head writes zeros into that head's slice of
+        // every row of the user (also rows past the grid when the user is longer than max_seqlen)
+        pdl_wait_primary();
+        if (qblk == 0) {
+            if (h == 0 && threadIdx.x == 0)
+                set_flag(a.ws, g.flags);
+            for (int64_t x = threadIdx.x; x < (int64_t)g.N * (kTcD / 4); x += kTcThreads) {
+                const int64_t r = x / (kTcD / 4);
+                const int c4 = (int)(x % (kTcD / 4));
+                reinterpret_cast<float4*>(part + (g.tok0 + r) * HD + (int64_t)h * kTcD)[c4] =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+        pdl_launch_dependents();
+        return;
+    }
     if (qrow0 >= g.N) {
         pdl_launch_dependents();
         return;                                               // no queries here (uniform)
     }
 
-    const int32_t i0 = g.C + qrow0;                           // absolute position of row 0
+    const int32_t i0 = qrow0;                                 // position of row 0
     const int32_t last_q = min(g.N, qrow0 + kTile) - 1;
-    const int32_t kend = min(g.L, g.C + last_q + 1);          // later keys are never visible
-    const int32_t ct = kPaged ? (g.C + kTile - 1) / kTile : 0;
-    const int32_t nnew = kend > g.C ? (kend - g.C + kTile - 1) / kTile : 0;
-    const int32_t ntot = ct + nnew;
-    const int32_t t_begin = (int32_t)(((int64_t)ntot * split) / nsplit);
-    const int32_t t_end = (int32_t)(((int64_t)ntot * (split + 1)) / nsplit);
-    const int32_t n = g.ok ? t_end - t_begin : 0;
-    const int64_t HD = (int64_t)a.H * kTcD;
-    float* part = a.part + (int64_t)split * a.total_tokens * HD;
-    // the LayerNorm kernel sums this many partial planes for each of these tokens (written once
-    // the kernel before this one -- possibly the previous call's LayerNorm kernel, which reads
-    // the same workspace -- has finished)
-    auto write_counts = [&]() {
-        if (kPaged && h == 0 && split == 0)
-            for (int r = threadIdx.x; r < kTile; r += kTcThreads)
-                if (qrow0 + r < g.N)
-                    a.counts[g.tok0 + qrow0 + r] = g.ok ? nsplit : 1;
-    };
-
-    if (n <= 0) {
-        pdl_wait_primary();
-        write_counts();
-        // nothing to accumulate: this split's partial rows are zero
-        for (int x = threadIdx.x; x < kTile * (kTcD / 4); x += kTcThreads) {
-            const int r = x / (kTcD / 4), c4 = x % (kTcD / 4);
-            if (qrow0 + r < g.N)
-                reinterpret_cast<float4*>(part + (g.tok0 + qrow0 + r) * HD + (int64_t)h * kTcD)[c4] =
-                    make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        pdl_launch_dependents();
-        return;
-    }
+    const int32_t kend = min(g.L, last_q + 1);                // later keys are never visible
+    const int n = (kend + kTile - 1) / kTile;                 // key tiles (>= 1)
 
     // ---------------------------------------------------------------- shared memory carve-up
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -429,12 +237,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* win = reinterpret_cast<float*>(smem + kOffWin);
     int32_t* s_bounds = reinterpret_cast<int32_t*>(smem + kOffBounds);
     float* s_rab = reinterpret_cast<float*>(smem + kOffRab);
-    int32_t* s_pages = reinterpret_cast<int32_t*>(smem + kOffPages);
-
-    // cached logical pages this CTA reads: [lp_begin, lp_end)
-    const int P = kPaged ? a.P : 1;
-    const int32_t lp_begin = kPaged ? (t_begin < ct ? t_begin * (kTile / P) : 0) : 0;
-    const int32_t lp_end = kPaged ? (t_begin < ct ? min(min(t_end, ct) * (kTile / P), (g.C + P - 1) / P) : 0) : 0;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -462,19 +264,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 2 || warp == 3) {
-        const int ht = threadIdx.x - 64;
-        if (kPaged) {
-            // validate the staged page ids this CTA will use (-1 = skip the load)
-            for (int k = lp_begin + ht; k < lp_end && k < kMaxPageIds; k += 64) {
-                const int32_t pg = s_pages[k];
-                if (pg < 0 || pg >= a.num_pages) {
-                    set_flag(a.ws, HSTU_DEV_BAD_PAGE);
-                    s_pages[k] = -1;
-                }
-            }
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -484,22 +273,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // are touched only after the previous kernel on the stream has finished (a no-op unless
     // this grid was launched as a programmatic dependent)
     pdl_wait_primary();
-    write_counts();
 
     if ((warp == 0 || warp == 3) && lane == 0) {
         // ============================================================ TMA producers
-        // warp 0 loads Q and the K tiles, warp 3 the V tiles: a single thread issuing every
-        // page box of a paged tile would serialise on TMA issue latency.
+        // warp 0 loads Q and the K tiles, warp 3 the V tiles
         const bool is_v = warp == 3;
         uint64_t* full = is_v ? v_full : k_full;
         uint64_t* empty = is_v ? v_empty : k_empty;
         const int stages = is_v ? kVStages : kKStages;
         const uint32_t ring = sbase + (is_v ? kOffV : kOffK);
         const CUtensorMap* tm_rows = is_v ? &tm_v : &tm_k;
-        const CUtensorMap* tm_pages = is_v ? &tm_vp : &tm_kp;
         tma_prefetch_desc(tm_rows);
-        if (kPaged)
-            tma_prefetch_desc(tm_pages);
         if (!is_v) {
             tma_prefetch_desc(&tm_q);
             mbar_arrive_expect_tx(q_full, kTileBytes);
@@ -508,48 +292,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         int issued = 0;
         for (int t = 0; t < n; ++t) {
-            const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
+            const TileGeo tg = tile_geo(t, g.L);
             const int st = t % stages;
             // tile t goes into stage t % stages once the MMA that read tile t - stages is done
             if (t >= stages && !mbar_wait(&empty[st], ((t / stages) & 1) ^ 1, abort_flag, tmo))
                 break;
             const uint32_t dst = ring + st * kTileBytes;
-            if (kPaged && tg.cached) {
-                // gather: one box of P rows per cached page and channel half
-                const int lp0 = tg.j0 / P;
-                const int npg = kTile / P;
-                int32_t pages[kTile / 8];
-                uint32_t bytes = 0;
-                for (int k = 0; k < npg; ++k) {
-                    const int lp = lp0 + k;
-                    int32_t pg = -1;
-                    if (lp < lp_end) {
-                        if (lp < kMaxPageIds) {
-                            pg = s_pages[lp];
-                        } else {
-                            pg = a.page_table[(int64_t)b * a.max_pages + lp];
-                            if (pg < 0 || pg >= a.num_pages) {
-                                set_flag(a.ws, HSTU_DEV_BAD_PAGE);
-                                pg = -1;
-                            }
-                        }
-                        if (pg >= 0)
-                            bytes += (uint32_t)P * 128u * 2u;
-                    }
-                    pages[k] = pg;
-                }
-                mbar_arrive_expect_tx(&full[st], bytes);
-                for (int k = 0; k < npg; ++k)
-                    if (pages[k] >= 0)
-                        for (int hf = 0; hf < 2; ++hf)
-                            tma_load_2d(tm_pages, dst + hf * kHalf + k * P * 128, &full[st], hf * 64,
-                                        (pages[k] * a.H + h) * P);
-            } else {
-                const int32_t row = (int32_t)(g.key_row0 + (tg.j0 - g.C));
-                mbar_arrive_expect_tx(&full[st], kTileBytes);
-                for (int hf = 0; hf < 2; ++hf)
-                    tma_load_3d(tm_rows, dst + hf * kHalf, &full[st], hf * 64, h, row);
-            }
+            const int32_t row = (int32_t)(g.key_row0 + tg.j0);
+            mbar_arrive_expect_tx(&full[st], kTileBytes);
+            for (int hf = 0; hf < 2; ++hf)
+                tma_load_3d(tm_rows, dst + hf * kHalf, &full[st], hf * 64, h, row);
             issued = t + 1;
         }
         // drain: loads still in flight must land before the CTA may exit (a local flag, so
@@ -643,7 +395,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (!ok)
                     break;
             }
-            const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
+            const TileGeo tg = tile_geo(t, g.L);
             const int32_t dist0 = i0 - tg.j0 + (kTile - 1);       // distance at window index 0
             float* wbuf = win + wb * (kWinBuf / 4);
             int32_t d[8];
@@ -689,7 +441,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int t = 0; t < n; ++t) {
             const int vst = t % kVStages;
             const int sb = t & 1;
-            const TileGeo tg = tile_geo(t_begin + t, ct, g.C, g.L);
+            const TileGeo tg = tile_geo(t, g.L);
             ok = ok && mbar_wait_warp(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
             ok = ok && mbar_wait_warp(&win_full[sb], (t >> 1) & 1, abort_flag, tmo);
             if (!ok)
@@ -699,7 +451,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const bool full = (qrow0 + kTile - 1 < g.N) && (tg.j0 + kTile - 1 < tg.kvend) &&
                               (tg.j0 + kTile - 1 <= i0) && (tg.j0 + kTile - 1 < g.hist);
             const int32_t lim = min(lim_row, tg.kvend);
-            const int32_t diag = (row_valid && !tg.cached) ? i_abs : -1;
+            const int32_t diag = row_valid ? i_abs : -1;
             const int jc0 = tg.j0 + wg * 64;                  // key position of column 0 of this half
             const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0) + wg * 64;
             uint32_t sv[32], sv2[32];
@@ -800,33 +552,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
-void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
-                    cudaStream_t stream)
+void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, int32_t B, cudaStream_t stream)
 {
     if (B <= 0 || a.qblocks <= 0)
         return;
-    // the shared-memory opt-in is a per-device setting of each kernel
+    // the shared-memory opt-in is a per-device setting of the kernel
     static std::atomic<uint32_t> attr_set[64];
     int dev = 0;
     cudaGetDevice(&dev);
-    const uint32_t bit = paged ? 2u : 1u;
-    if (dev < 0 || dev >= 64 || !(attr_set[dev].load(std::memory_order_relaxed) & bit)) {
-        if (paged)
-            cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        else
-            cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_relaxed)) {
+        cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (dev >= 0 && dev < 64)
-            attr_set[dev].fetch_or(bit, std::memory_order_relaxed);
+            attr_set[dev].store(1, std::memory_order_relaxed);
     }
-    // paged: one CTA per piece of the balanced plan; the plan sizes its pieces to fit
-    // max(one per SM, one per (entry, head)) CTAs, and CTAs past the last piece exit at once.
-    // Jagged: (head, user) x query block.
-    const int64_t entries = (int64_t)B * a.qblocks;
-    const int64_t paged_grid = entries * a.H > a.target_ctas ? entries * a.H : a.target_ctas;
-    dim3 grid = paged ? dim3((unsigned)paged_grid, 1, 1)
-                      : dim3((unsigned)((int64_t)a.H * B), (unsigned)a.qblocks, 1);
+    // (head, user) x query block
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
+    cfg.gridDim = dim3((unsigned)((int64_t)a.H * B), (unsigned)a.qblocks, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
@@ -835,10 +576,7 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.overlap_previous ? 1 : 0;          // programmatic dependent launch on request
-    if (paged)
-        cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
-    else
-        cudaLaunchKernelEx(&cfg, attn_tc_kernel<false>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
+    cudaLaunchKernelEx(&cfg, attn_tc_kernel, m.q, m.k, m.v, bb, a);
 }
 
 }  // namespace hstu

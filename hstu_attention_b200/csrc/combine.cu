@@ -51,6 +51,9 @@ ln_gate_kernel(const float* __restrict__ part, int32_t S_all, const int32_t* __r
                int32_t HD, const T* __restrict__ u, T* __restrict__ out, float eps)
 {
     using V = typename Vec4<T>::type;
+    // the next attention call (a programmatic dependent of this grid) may start its set-up now;
+    // it waits for this grid's completion before it touches anything this grid reads or writes
+    sm100::pdl_launch_dependents();
     sm100::pdl_wait_primary();          // launched early behind the attention grid
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);
@@ -127,6 +130,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 ln_gate_kernel_scalar(const float* __restrict__ part, int32_t S_all, const int32_t* __restrict__ counts,
                       int64_t ntok, int32_t HD, const T* __restrict__ u, T* __restrict__ out, float eps)
 {
+    sm100::pdl_launch_dependents();
     sm100::pdl_wait_primary();
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);

@@ -79,39 +79,40 @@ __device__ __forceinline__ int64_t warp_prefix_offset(const int32_t* lens, int b
 }
 
 // Per-user geometry shared by the attention kernels.  For the jagged layout the queries
-// are all L tokens (q_begin = 0); for the paged layout they are the N new tokens placed
-// after C cached ones.
+// are all L tokens; for the paged layout they are the N new tokens placed after C cached ones.
+// The helpers only read the length arrays: a rejected user's status bits are returned in
+// `flags`, and the kernel raises them once it may write the workspace.
 struct UserGeom {
     int64_t tok0;      // first query token row in the q/u/out arrays
     int64_t key_row0;  // first row of this user's non-cached keys in k/v (or k_new/v_new)
     int32_t C;         // cached keys read from pages (0 for jagged)
-    int32_t N;         // query tokens (jagged: L)
+    int32_t N;         // query tokens (jagged: L); rows that cannot be located count as 0
     int32_t L;         // total keys = C + N
     int32_t hist;      // L - num_targets
+    uint32_t flags;    // HSTU_DEV_* bits of a rejected user (0 when ok)
     bool ok;
 };
 
-// Jagged geometry with validation; sets status bits and returns ok = false for a bad user.
+// Jagged geometry with validation.
 __device__ __forceinline__ UserGeom jagged_geom(const int32_t* seq_offsets, const int32_t* num_targets,
-                                                int b, int64_t total_tokens, int32_t max_seqlen,
-                                                int32_t n_max, void* ws, bool report)
+                                                int b, int64_t total_tokens, int32_t max_seqlen, int32_t n_max)
 {
     UserGeom g;
     int64_t s0 = seq_offsets[b], s1 = seq_offsets[b + 1];
     int32_t T = num_targets ? num_targets[b] : 0;
     int64_t L = s1 - s0;
     g.ok = true;
+    g.flags = 0;
     if (s0 < 0 || s1 > total_tokens || L < 0 || T < 0 || T > L || L > max_seqlen) {
-        if (report) set_flag(ws, HSTU_DEV_BAD_LENGTH);
+        g.flags = HSTU_DEV_BAD_LENGTH;
         g.ok = false;
     } else if (L > n_max) {
-        if (report) set_flag(ws, HSTU_DEV_BAD_NMAX);
+        g.flags = HSTU_DEV_BAD_NMAX;
         g.ok = false;
     }
     g.tok0 = s0;
     g.key_row0 = s0;
     g.C = 0;
-    // rows that cannot be located inside [0, total_tokens) are never written
     g.N = (s0 < 0 || s1 > total_tokens || L < 0) ? 0 : (int32_t)L;
     g.L = g.N;
     g.hist = g.N - (T > 0 && T <= g.N ? T : 0);
@@ -121,19 +122,19 @@ __device__ __forceinline__ UserGeom jagged_geom(const int32_t* seq_offsets, cons
 // Paged geometry; must be called by a full warp (prefix sum of new_lens).
 __device__ __forceinline__ UserGeom paged_geom(const int32_t* cached_lens, const int32_t* new_lens,
                                                const int32_t* num_targets, int b, int64_t total_new,
-                                               int32_t max_new, int32_t max_cached, int32_t n_max,
-                                               void* ws, bool report)
+                                               int32_t max_new, int32_t max_cached, int32_t n_max)
 {
     UserGeom g;
     int64_t off = warp_prefix_offset(new_lens, b);
     int32_t C = cached_lens[b], N = new_lens[b];
     int32_t T = num_targets ? num_targets[b] : 0;
     g.ok = true;
+    g.flags = 0;
     if (C < 0 || N < 0 || T < 0 || T > N || N > max_new || C > max_cached || off + N > total_new) {
-        if (report) set_flag(ws, HSTU_DEV_BAD_LENGTH);
+        g.flags = HSTU_DEV_BAD_LENGTH;
         g.ok = false;
     } else if ((int64_t)C + N > n_max) {
-        if (report) set_flag(ws, HSTU_DEV_BAD_NMAX);
+        g.flags = HSTU_DEV_BAD_NMAX;
         g.ok = false;
     }
     g.tok0 = off;
@@ -142,7 +143,6 @@ __device__ __forceinline__ UserGeom paged_geom(const int32_t* cached_lens, const
     g.N = N > 0 ? N : 0;
     g.L = g.C + g.N;
     g.hist = g.L - (T > 0 ? T : 0);
-    // an unlocatable user (rows past total_new) must not be written at all
     if (off + g.N > total_new)
         g.N = 0;
     return g;

@@ -45,6 +45,10 @@ struct TcArgs {
     int32_t overlap_previous;   // paged: launched as a programmatic dependent of the previous kernel
 };
 
+// The paged tensor-core kernel (attn_paged.cu) takes the same argument block; seq_offsets and
+// target_ctas are unused there.
+using PagedArgs = TcArgs;
+
 struct TcMaps {
     CUtensorMap q, k, v, kp, vp;
 };
@@ -78,6 +82,7 @@ struct BwdArgs {
     float* drab;                           // [H][NB] fp32, accumulated (zeroed by the caller)
     int64_t total_tokens;
     int32_t B, H, D, NB, n_max;
+    int32_t max_seqlen;                    // users longer than this are rejected (as in the forward)
     double ln_nmax;
     float inv_n;
 };
@@ -86,7 +91,11 @@ void launch_jagged_bwd(const BwdArgs& a, const float* o, const void* u, const vo
                        bool fp32, cudaStream_t stream);
 
 void launch_attn_simt(const SimtArgs& a, bool paged, bool fp32, int32_t B, cudaStream_t stream);
-void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, bool paged, int32_t B,
-                    cudaStream_t stream);
+// Jagged prefill on tensor cores (bf16, D = 128).
+void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, int32_t B, cudaStream_t stream);
+// Paged cache hit on tensor cores (bf16, D = 128); at most paged_max_users() users per call.
+void launch_attn_paged(const TcMaps& m, const PagedArgs& a, const BucketBounds& bb, int num_sms,
+                       cudaStream_t stream);
+int paged_max_users();
 
 }  // namespace hstu

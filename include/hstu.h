@@ -72,8 +72,7 @@ enum {
                                         appended position beyond max_pages_per_user * P,
                                         or a length above the bound passed on the host */
     HSTU_DEV_BAD_NMAX = 1u << 2,     /* a user's total length exceeds n_max */
-    HSTU_DEV_TIMEOUT = 1u << 3,      /* an in-kernel wait gave up (kernel returned early) */
-    HSTU_DEV_SMEM_ALIGN = 1u << 4    /* shared memory not aligned as the kernel requires */
+    HSTU_DEV_TIMEOUT = 1u << 3       /* an in-kernel wait gave up (kernel returned early) */
 };
 
 typedef struct {
@@ -97,7 +96,7 @@ typedef struct {
  * launched with programmatic dependent launch, so its set-up -- the work plan from the length
  * arrays, the page-table reads, barrier and tensor-memory set-up -- may run while the kernel
  * enqueued before it on the same stream is still finishing.  It waits for that kernel before it
- * reads q/k/v/u, the pages or rab and before it writes anything but the status word.  Set the
+ * reads q/k/v/u, the pages or rab and before it writes anything, the status word included.  Set the
  * bit only when the kernel enqueued right before the call does not write seq_offsets,
  * page_table, cached_lens, new_lens or num_targets (for example when consecutive layers run back
  * to back, or when the metadata was copied from the host).  Without the bit the call starts

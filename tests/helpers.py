@@ -101,16 +101,17 @@ def paged_params(hb, c: gen.PagedCase):
                      max_pages_per_user=c.max_pages, ln_eps=c.eps)
 
 
-def gpu_paged(hb, c: gen.PagedCase, pool=None, ws=None, page_table=None, poison=False):
+def gpu_paged(hb, c: gen.PagedCase, pool=None, ws=None, page_table=None, poison=False, max_new=None):
     import torch
 
     p = paged_params(hb, c)
     kp, vp = pool if pool is not None else device_pool(c, poison=poison)
+    mn = int(max_new if max_new is not None else max(c.max_new, 1))
     if ws is None:
-        ws = hb.Workspace(p, c.B, max(c.Tn, 1), max(c.max_new, 1))
+        ws = hb.Workspace(p, c.B, max(c.Tn, 1), mn)
     pt = dev(c.page_table if page_table is None else page_table)
     o = hb.paged_fwd(p, dev(c.q_new), dev(c.k_new), dev(c.v_new), dev(c.u_new), kp, vp, pt, dev(c.cached_lens),
-                     dev(c.new_lens), dev(c.num_targets), dev(c.rab), max_new=max(c.max_new, 1), workspace=ws)
+                     dev(c.new_lens), dev(c.num_targets), dev(c.rab), max_new=mn, workspace=ws)
     torch.cuda.synchronize()
     return o, ws, p, (kp, vp)
 

@@ -70,6 +70,25 @@ def test_bwd_rejected_user_has_zero_gradients(cuda_lib):
         _close(g[10:], r, 1e-2, f"valid user {name}")
 
 
+def test_bwd_user_longer_than_max_seqlen(cuda_lib):
+    """The forward rejects a user longer than max_seqlen (its o is zero); the backward must too:
+    zero dq/dk/dv/du for that user and a drab that holds only the valid users' pairs."""
+    hb = cuda_lib
+    c = gen.jagged_case([60, 300, 45], [4, 64, 5], H=4, D=128, NB=64, n_max=512, dtype="bf16", seed=23)
+    dout = _dout(c, 8)
+    got, status = _run(hb, c, dout, 129)
+    assert status & hb.DEV_BAD_LENGTH
+    for g in got[:4]:
+        assert not np.any(g[60:360])                  # dq, dk, dv, du of the rejected user
+    keep = np.r_[0:60, 360:405]
+    off = np.array([0, 60, 105])
+    ref = oracle.hstu_jagged_bwd(c.q[keep], c.k[keep], c.v[keep], c.u[keep], dout[keep], off, c.num_targets[[0, 2]],
+                                 c.rab, c.n_max, c.eps)
+    for name, g, r in zip(NAMES[:4], got[:4], ref[:4]):
+        _close(g[keep], r, 1e-2, f"valid users {name}")
+    _close(got[4], ref[4], 1e-2, "drab of the valid users only")
+
+
 def test_bwd_empty_batch_zeroes_drab(cuda_lib):
     import torch
 

@@ -288,6 +288,34 @@ def test_device_flags_bad_page_and_lengths(cuda_lib):
     assert_close(host(o3)[10:], ref, "bf16", "valid user next to a rejected one")
 
 
+def test_user_longer_than_the_host_bound_is_zeroed(cuda_lib):
+    """A user longer than max_seqlen (jagged) or with more than max_new new tokens (paged) is
+    rejected: BAD_LENGTH, and every one of its output rows is zero -- also the rows past the
+    query blocks the host bound sized the grid for.  The other users are unaffected."""
+    hb = cuda_lib
+    jc = gen.jagged_case([60, 300, 45], [4, 64, 5], H=4, D=128, NB=64, n_max=512, dtype="bf16", seed=21)
+    o, ws, _ = gpu_jagged(hb, jc, max_seqlen=129)          # user 1 (300 tokens) is over the bound
+    assert ws.status() & hb.DEV_BAD_LENGTH
+    out = gen.as_f32(host(o))
+    assert np.all(out[60:360] == 0.0)
+    for b in (0, 2):
+        s0, s1 = int(jc.seq_offsets[b]), int(jc.seq_offsets[b + 1])
+        ref = oracle.hstu_jagged(jc.q[s0:s1], jc.k[s0:s1], jc.v[s0:s1], jc.u[s0:s1], [0, s1 - s0],
+                                 jc.num_targets[b:b + 1], jc.rab, jc.n_max)
+        assert_close(host(o)[s0:s1], ref, "bf16", f"jagged user {b} next to a rejected one")
+    # paged: user 1 has 300 new tokens against max_new = 129
+    c = gen.paged_case([40, 100, 7], [0, 236, 3], [5, 64, 2], H=4, D=128, P=32, NB=64, n_max=512, num_pages=40,
+                       dtype="bf16", seed=22)
+    o2, ws2, _, _ = gpu_paged(hb, c, max_new=129)
+    assert ws2.status() & hb.DEV_BAD_LENGTH
+    out2 = gen.as_f32(host(o2))
+    off = c.new_offsets
+    assert np.all(out2[off[1]:off[2]] == 0.0)
+    ref = oracle_paged(c)
+    keep = np.r_[off[0]:off[1], off[2]:off[3]]
+    assert_close(host(o2)[keep], ref[keep], "bf16", "paged users next to a rejected one")
+
+
 def test_empty_calls_are_noops(cuda_lib):
     hb = cuda_lib
     import torch
@@ -333,48 +361,95 @@ def test_paged_full_size_one_layer(cuda_lib):
     assert_close(host(o), oracle_paged(c), "bf16", "paged layer 0")
 
 
-def test_long_history_sampled(cuda_lib):
-    """Long-history cache hit (32 users, cached U[8192,16384], 256 candidates, H=8, P=64)."""
+def test_long_history(cuda_lib):
+    """Long-history cache hit (32 users, cached U[8192,16384], 256 candidates, H=8, P=64): every
+    row of the shortest and of the longest user, plus rows sampled over the whole batch."""
     c = gen.config4_long()
     o, ws, _, _ = gpu_paged(cuda_lib, c)
     assert ws.status() == 0
-    rows = _sample_rows(c.Tn, 64, 4)
-    assert_close(host(o)[rows], oracle_paged(c, rows=rows), "bf16", "long history sampled")
+    off = np.concatenate([[0], np.cumsum(c.new_lens)])
+    rows = set(_sample_rows(c.Tn, 64, 4).tolist())
+    for b in (int(np.argmin(c.cached_lens)), int(np.argmax(c.cached_lens))):
+        rows |= set(range(int(off[b]), int(off[b + 1])))
+    rows = np.array(sorted(rows), dtype=np.int64)
+    assert_close(host(o)[rows], oracle_paged(c, rows=rows), "bf16", "long history")
 
 
-def test_mixed_batch_sampled(cuda_lib):
-    """Mixed serving batch: hits through the paged path (with their appends), misses through
-    jagged prefill followed by the append of their history into pages."""
+def _pages_to_host(kp, vp, ids):
+    """The listed physical pages of the pool, copied to the host (renumbered 0..len-1)."""
+    import torch
+
+    idx = torch.from_numpy(np.asarray(ids, dtype=np.int64)).cuda()
+    return host(kp.index_select(0, idx)).copy(), host(vp.index_select(0, idx)).copy()
+
+
+def _renumber(pt, ids):
+    """Page table over the compact host copy made by _pages_to_host(ids)."""
+    where = {int(x): i for i, x in enumerate(ids)}
+    return np.vectorize(lambda x: where.get(int(x), -1))(pt).astype(np.int32)
+
+
+def test_mixed_batch(cuda_lib):
+    """Mixed serving batch.  Hits: append of their new history tokens (byte-exact over every page
+    they touch) and paged attention (every output row).  Misses: jagged prefill (every row of the
+    smaller half of the users, sampled rows of the rest), then the append of their history into
+    pages (byte-exact over every page the misses own)."""
     import torch
 
     hb = cuda_lib
     hits, misses, miss_pt, miss_hist = gen.config5_mixed()
-    o_hit, ws, p, (kp, vp) = gpu_paged(hb, hits)
+    p = paged_params(hb, hits)
+    kp, vp = device_pool(hits)
+    ws = hb.Workspace(p, max(hits.B, misses.B), max(hits.Tn, misses.T), int(misses.max_seqlen))
+    hit_ids = np.unique(hits.page_table[hits.page_table >= 0])
+    before_k, before_v = _pages_to_host(kp, vp, hit_ids)
+
+    o_hit, _, _, _ = gpu_paged(hb, hits, pool=(kp, vp), ws=ws)
     assert ws.status() == 0
-    rows = _sample_rows(hits.Tn, 48, 5)
-    assert_close(host(o_hit)[rows], oracle_paged(hits, rows=rows), "bf16", "mixed hits")
-    o_miss, ws2, _ = gpu_jagged(hb, misses, max_seqlen=int(misses.max_seqlen))
-    assert ws2.status() == 0
+    assert_close(host(o_hit), oracle_paged(hits), "bf16", "mixed hits")
+
+    hb.kv_append(p, kp, vp, dev(hits.page_table), dev(hits.k_new), dev(hits.v_new), dev(hits.cached_lens),
+                 dev(hits.new_lens), dev(hits.num_targets), max_new=hits.max_new, workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    got_k, got_v = _pages_to_host(kp, vp, hit_ids)
+    cpt = _renumber(hits.page_table, hit_ids)
+    assert oracle.kv_append(before_k, before_v, cpt, hits.k_new, hits.v_new, hits.cached_lens, hits.new_offsets,
+                            hits.new_lens - hits.num_targets) == 0
+    assert np.array_equal(got_k.view(np.uint8), before_k.view(np.uint8))
+    assert np.array_equal(got_v.view(np.uint8), before_v.view(np.uint8))
+
+    o_miss, _, _ = gpu_jagged(hb, misses, ws=ws, max_seqlen=int(misses.max_seqlen))
+    assert ws.status() == 0
     lens = misses.lengths
-    small = np.argsort(lens)[:8]                     # oracle time: the smaller users, all rows
+    small = np.argsort(lens, kind="stable")[: misses.B // 2]
     rows = np.concatenate([np.arange(misses.seq_offsets[b], misses.seq_offsets[b + 1]) for b in sorted(small)])
-    rows = np.concatenate([rows, _sample_rows(misses.T, 24, 6)])
-    rows = np.unique(rows)
+    big = np.argsort(lens, kind="stable")[misses.B // 2:]
+    for b in big:                                    # first, last, first candidate of each big user
+        s0, s1 = int(misses.seq_offsets[b]), int(misses.seq_offsets[b + 1])
+        rows = np.concatenate([rows, [s0, s0 + 127, s1 - int(misses.num_targets[b]), s1 - 1]])
+    rows = np.unique(np.concatenate([rows, _sample_rows(misses.T, 64, 6)]))
     assert_close(host(o_miss)[rows], oracle_jagged(misses, rows=rows), "bf16", "mixed misses")
-    # misses populate pages: append each miss's history (cached 0, candidates not appended)
+
+    # misses populate pages: append each miss's whole history (cached 0; candidates not appended)
+    miss_ids = np.unique(miss_pt[miss_pt >= 0])
+    assert not np.intersect1d(miss_ids, hit_ids).size
+    mk, mv = _pages_to_host(kp, vp, miss_ids)
     pm = hb.params(4, 128, torch.bfloat16, 128, hits.n_max, page_size=32, num_pages=hits.num_pages,
                    max_pages_per_user=miss_pt.shape[1])
-    zeros = np.zeros(64, dtype=np.int32)
+    zeros = np.zeros(misses.B, dtype=np.int32)
     hb.kv_append(pm, kp, vp, dev(miss_pt), dev(misses.k), dev(misses.v), dev(zeros), dev(misses.lengths),
                  dev(misses.num_targets), max_new=int(misses.max_seqlen), workspace=ws)
     torch.cuda.synchronize()
     assert ws.status() == 0
-    for b in [int(small[0]), int(np.argmax(lens))]:
-        s0 = int(misses.seq_offsets[b])
-        for pos in [0, int(miss_hist[b]) - 1, int(miss_hist[b]) // 2]:
-            page = int(miss_pt[b, pos // 32])
-            got = host(kp[page, :, pos % 32, :])
-            assert np.array_equal(got, misses.k[s0 + pos])
+    got_k, got_v = _pages_to_host(kp, vp, miss_ids)
+    assert oracle.kv_append(mk, mv, _renumber(miss_pt, miss_ids), misses.k, misses.v, zeros, misses.seq_offsets,
+                            misses.lengths - misses.num_targets) == 0
+    assert np.array_equal(got_k.view(np.uint8), mk.view(np.uint8))
+    assert np.array_equal(got_v.view(np.uint8), mv.view(np.uint8))
+    # the hits' pages were not touched by the misses' append
+    again_k, _ = _pages_to_host(kp, vp, hit_ids)
+    assert np.array_equal(again_k.view(np.uint8), before_k.view(np.uint8))
 
 
 # --------------------------------------------------------------------------- launch overlap flag

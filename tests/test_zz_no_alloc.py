@@ -11,7 +11,8 @@ import numpy as np
 import pytest
 
 from hstu_attention_b200 import inputs as gen
-from tests.helpers import BF16_TOL, FP32_TOL, dev, device_pool, gpu_paged, host, paged_params, values
+from tests.helpers import (BF16_TOL, FP32_TOL, assert_close, dev, device_pool, gpu_paged, host, oracle_paged,
+                           paged_params, values)
 
 pytestmark = pytest.mark.gpu
 
@@ -68,6 +69,9 @@ def test_two_calls_in_a_row_match_the_workspace_entry(cuda_lib):
     _close(out_a, ref_a, "bf16", "cache-hit layer")
     _close(out_b, ref_b, "bf16", "small ragged batch")
     assert torch.equal(out_a.view(torch.int16), out_a2.view(torch.int16))   # deterministic on repeat
+    # and against the float64 oracle directly
+    assert_close(host(out_a), oracle_paged(a), "bf16", "no-alloc cache-hit layer vs oracle")
+    assert_close(host(out_b), oracle_paged(b), "bf16", "no-alloc ragged batch vs oracle")
 
 
 def test_fp32_path_matches_the_workspace_entry(cuda_lib):
@@ -85,6 +89,7 @@ def test_fp32_path_matches_the_workspace_entry(cuda_lib):
     assert int(f1.item()) == 0 and int(f2.item()) == 0
     _close(o1, ref, "fp32", "tiny fp32, first call")
     _close(o2, ref, "fp32", "tiny fp32, second call")
+    assert_close(host(o2), oracle_paged(c), "fp32", "no-alloc tiny fp32 vs oracle")
 
 
 def test_flags_are_per_call(cuda_lib):
