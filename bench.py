@@ -17,6 +17,7 @@ read ~340 MB of distinct pages and tokens per step, more than the 126 MB L2, so 
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -268,12 +269,12 @@ def bench_prefill(hb, device, steps, warmup, peaks):
     p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max, flags=hb.FLAG_OVERLAP_PREVIOUS)
     ws = hb.Workspace(p, c.B, c.T, 4096, device=device)
     out = torch.empty_like(q)
-    # rotate inputs larger than L2: two copies of q/k/v/u (2 x 71 MB) alternate
-    q2, k2, v2, u2 = q.clone(), k.clone(), v.clone(), u.clone()
-    sets = [(q, k, v, u), (q2, k2, v2, u2)]
+    # rotate three copies of q/k/v/u (3 x 83 MB, more than the 126 MB L2) so that each timed call
+    # reads its inputs from HBM
+    sets = [(q, k, v, u)] + [(q.clone(), k.clone(), v.clone(), u.clone()) for _ in range(2)]
     stream = torch.cuda.current_stream()
     for i in range(warmup):
-        a = sets[i % 2]
+        a = sets[i % len(sets)]
         hb.jagged_fwd(p, *a, off, nt, rab, max_seqlen=4096, workspace=ws, out=out)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -287,7 +288,7 @@ def bench_prefill(hb, device, steps, warmup, peaks):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / (2 * steps)
+    ms = e0.elapsed_time(e1) / (len(sets) * steps)
     pairs = 0
     for L, T in zip(c.lengths, c.num_targets):
         hist = int(L - T)
@@ -302,6 +303,207 @@ def bench_prefill(hb, device, steps, warmup, peaks):
                          "traffic": PREFILL_TRAFFIC_BYTES if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None,
                          "traffic_kernel": "attn_tc_kernel (jagged) per launch"},
             "launches_per_call": 2}
+
+
+def _to_dev(x, device):
+    import torch
+
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    if x.dtype == np.int64:
+        x = x.astype(np.int32)
+    return torch.from_numpy(x).to(device)
+
+
+def paged_pairs(c) -> int:
+    """Unmasked (query, key) pairs per head of a paged call."""
+    pairs = 0
+    for C, N, T in zip(c.cached_lens, c.new_lens, c.num_targets):
+        C, N, T = int(C), int(N), int(T)
+        hist = C + N - T
+        q = np.arange(C, C + N)
+        pairs += int(np.sum(np.where(q < hist, q + 1, hist + 1)))
+    return pairs
+
+
+def jagged_pairs(lengths, targets) -> int:
+    pairs = 0
+    for L, T in zip(lengths, targets):
+        hist = int(L) - int(T)
+        pairs += hist * (hist + 1) // 2 + int(T) * (hist + 1)
+    return pairs
+
+
+def graph_ms(graph, steps, stream) -> float:
+    """Mean ms per replay of `graph` over `steps` replays (CUDA events on `stream`)."""
+    import torch
+
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def bench_long_history(hb, device, steps, warmup, peaks, with_cpu):
+    """Sub-line: the long-history cache hit (32 users, cached U[8192,16384], 256 candidates,
+    H=8, P=64): one paged call per step, 1.69 GB of distinct pages (more than L2)."""
+    import torch
+
+    c = gen.config4_long()
+    p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max, page_size=c.P, num_pages=c.num_pages,
+                  max_pages_per_user=c.max_pages, flags=hb.FLAG_OVERLAP_PREVIOUS)
+    shape = (c.num_pages, c.H, c.P, c.D)
+    kp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    vp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    ids = torch.from_numpy(c.page_ids.astype(np.int64)).to(device)
+    kp[ids] = _to_dev(c.pool_k, device)
+    vp[ids] = _to_dev(c.pool_v, device)
+    t = [_to_dev(x, device) for x in (c.q_new, c.k_new, c.v_new, c.u_new)]
+    meta = [_to_dev(x, device) for x in (c.page_table, c.cached_lens, c.new_lens, c.num_targets, c.rab)]
+    ws = hb.Workspace(p, c.B, c.Tn, c.max_new, device=device)
+    out = torch.empty_like(t[0])
+    for _ in range(warmup):
+        hb.paged_fwd(p, *t, kp, vp, *meta, max_new=c.max_new, workspace=ws, out=out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        hb.paged_fwd(p, *t, kp, vp, *meta, max_new=c.max_new, workspace=ws, out=out)
+    ms = graph_ms(g, steps, torch.cuda.current_stream())
+    assert ws.status() == 0
+    HD = c.H * c.D
+    pages = int(np.sum((c.cached_lens + c.P - 1) // c.P))
+    nbytes = int(np.sum(c.cached_lens)) * HD * 2 * 2 + c.Tn * HD * 2 * 5 + pages * 4
+    flops = 4 * c.D * c.H * paged_pairs(c)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tf = flops / (ms * 1e-3) / 1e12
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    bf16 = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    line = {"workload": "long-history cache hit: 32 users, cached U[8192,16384] (seed 1004), 256 candidates, "
+                        "H=8, D=128, P=64, NB=256, n_max=16640; one paged call per step",
+            "new_tokens": int(c.Tn), "ms_per_call": ms, "new_tokens_per_s": c.Tn / (ms * 1e-3),
+            "algorithmic_bytes_per_call": nbytes, "flops_per_call": flops,
+            "roofline": {"bound": "hbm and tensor (at the ridge)", "achieved_gbs": gbs, "hbm_peak_gbs": hbm,
+                         "hbm_frac": gbs / hbm, "achieved_tflops": tf, "bf16_peak_tflops": bf16,
+                         "tensor_frac": tf / bf16, "frac": max(gbs / hbm, tf / bf16)},
+            "l2": "inputs larger than L2 (1.69 GB of distinct pages per call)"}
+    if with_cpu:
+        import oracle
+
+        # seeded subset: the first user's 256 rows, extrapolated by unmasked pairs
+        sub = dataclasses.replace(c, cached_lens=c.cached_lens[:1], new_lens=c.new_lens[:1],
+                                  num_targets=c.num_targets[:1], page_table=c.page_table[:1])
+        ck, cv, cpt = sub.compact_pool()
+        nthreads = oracle.default_threads()
+        t0 = time.perf_counter()
+        oracle.hstu_paged(sub.q_new[:int(sub.Tn)], sub.k_new[:int(sub.Tn)], sub.v_new[:int(sub.Tn)],
+                          sub.u_new[:int(sub.Tn)], ck, cv, cpt, sub.cached_lens, sub.new_lens, sub.num_targets,
+                          sub.rab, sub.n_max, sub.eps, nthreads=nthreads)
+        dt = time.perf_counter() - t0
+        scale = paged_pairs(c) / max(1, paged_pairs(sub))
+        line["cpu_baseline"] = {"value": c.Tn / (dt * scale), "unit": "new tokens/s", "cores": nthreads,
+                                "kind": "oracle", "sample": f"user 0 only (256 rows, {dt:.2f} s), extrapolated "
+                                                            f"to the whole call by unmasked pairs (x{scale:.1f})"}
+    del kp, vp, ws, g
+    torch.cuda.empty_cache()
+    return line
+
+
+def bench_mixed(hb, device, steps, warmup, peaks, with_cpu):
+    """Sub-line: the mixed serving batch as one step -- the 64 hits append their new history
+    tokens and run the paged cache hit; the 64 misses run jagged prefill of history plus
+    candidates and then append their history into pages (one shared 262,144-page pool)."""
+    import torch
+
+    hits, misses, miss_pt, miss_hist = gen.config5_mixed()
+    flags = hb.FLAG_OVERLAP_PREVIOUS
+    ph = hb.params(hits.H, hits.D, torch.bfloat16, hits.NB, hits.n_max, page_size=hits.P, num_pages=hits.num_pages,
+                   max_pages_per_user=hits.max_pages, flags=flags)
+    pm = hb.params(hits.H, hits.D, torch.bfloat16, hits.NB, hits.n_max, page_size=hits.P, num_pages=hits.num_pages,
+                   max_pages_per_user=int(miss_pt.shape[1]), flags=flags)
+    pj = hb.params(misses.H, misses.D, torch.bfloat16, misses.NB, misses.n_max, flags=flags)
+    shape = (hits.num_pages, hits.H, hits.P, hits.D)
+    kp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    vp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    ids = torch.from_numpy(hits.page_ids.astype(np.int64)).to(device)
+    kp[ids] = _to_dev(hits.pool_k, device)
+    vp[ids] = _to_dev(hits.pool_v, device)
+    ht = [_to_dev(x, device) for x in (hits.q_new, hits.k_new, hits.v_new, hits.u_new)]
+    hmeta = [_to_dev(x, device) for x in (hits.page_table, hits.cached_lens, hits.new_lens, hits.num_targets)]
+    hrab = _to_dev(hits.rab, device)
+    mt = [_to_dev(x, device) for x in (misses.q, misses.k, misses.v, misses.u)]
+    moff, mnt, mrab = (_to_dev(x, device) for x in (misses.seq_offsets, misses.num_targets, misses.rab))
+    mpt, mzero, mlen = (_to_dev(x, device) for x in (miss_pt, np.zeros(misses.B, np.int32), misses.lengths))
+    max_seq = int(misses.max_seqlen)
+    ws = hb.Workspace(ph, max(hits.B, misses.B), max(hits.Tn, misses.T), max(hits.max_new, max_seq), device=device)
+    hout, mout = torch.empty_like(ht[0]), torch.empty_like(mt[0])
+
+    def step():
+        hb.kv_append(ph, kp, vp, hmeta[0], ht[1], ht[2], hmeta[1], hmeta[2], hmeta[3], max_new=hits.max_new,
+                     workspace=ws)
+        hb.paged_fwd(ph, *ht, kp, vp, *hmeta, hrab, max_new=hits.max_new, workspace=ws, out=hout)
+        hb.jagged_fwd(pj, *mt, moff, mnt, mrab, max_seqlen=max_seq, workspace=ws, out=mout)
+        hb.kv_append(pm, kp, vp, mpt, mt[1], mt[2], mzero, mlen, mnt, max_new=max_seq, workspace=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    ms = graph_ms(g, steps, torch.cuda.current_stream())
+    assert ws.status() == 0
+    tokens = int(hits.Tn + misses.T)
+    hit_flops = 4 * hits.D * hits.H * paged_pairs(hits)
+    miss_flops = 4 * misses.D * misses.H * jagged_pairs(misses.lengths, misses.num_targets)
+    tf = (hit_flops + miss_flops) / (ms * 1e-3) / 1e12
+    bf16 = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    line = {"workload": "mixed serving batch (seed 1005): 128 users, history lognormal(ln 2000, 1) clipped "
+                        "[64, 32768], candidates U[16,512]; 64 hits (append 8-32 + paged attention), 64 misses "
+                        "(jagged prefill + append of the history), H=4, D=128, P=32, 262,144-page pool",
+            "tokens": tokens, "hit_new_tokens": int(hits.Tn), "miss_tokens": int(misses.T), "ms_per_step": ms,
+            "tokens_per_s": tokens / (ms * 1e-3), "flops_per_step": hit_flops + miss_flops, "tflops": tf,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16},
+            "launches_per_step": 6, "l2": "inputs larger than L2 (about 2.1 GB of pages and tokens per step)"}
+    if with_cpu:
+        import oracle
+
+        # seeded subset: the two shortest hits (paged oracle) and the two shortest misses (prefill
+        # oracle), extrapolated to the whole step by unmasked pairs
+        nthreads = oracle.default_threads()
+        hsel = np.argsort(hits.cached_lens, kind="stable")[:2]
+        msel = np.argsort(misses.lengths, kind="stable")[:2]
+        t0 = time.perf_counter()
+        pairs_done = 0
+        for b in hsel:
+            o0, o1 = int(hits.new_offsets[b]), int(hits.new_offsets[b + 1])
+            sub = dataclasses.replace(hits, cached_lens=hits.cached_lens[b:b + 1], new_lens=hits.new_lens[b:b + 1],
+                                      num_targets=hits.num_targets[b:b + 1], page_table=hits.page_table[b:b + 1])
+            ck, cv, cpt = sub.compact_pool()
+            oracle.hstu_paged(hits.q_new[o0:o1], hits.k_new[o0:o1], hits.v_new[o0:o1], hits.u_new[o0:o1], ck, cv,
+                              cpt, sub.cached_lens, sub.new_lens, sub.num_targets, hits.rab, hits.n_max, hits.eps,
+                              nthreads=nthreads)
+            pairs_done += paged_pairs(sub) * hits.H
+        for b in msel:
+            s0, s1 = int(misses.seq_offsets[b]), int(misses.seq_offsets[b + 1])
+            oracle.hstu_jagged(misses.q[s0:s1], misses.k[s0:s1], misses.v[s0:s1], misses.u[s0:s1], [0, s1 - s0],
+                               misses.num_targets[b:b + 1], misses.rab, misses.n_max, misses.eps)
+            pairs_done += jagged_pairs([s1 - s0], [misses.num_targets[b]]) * misses.H
+        dt = time.perf_counter() - t0
+        scale = (hit_flops + miss_flops) / (4 * hits.D) / max(1, pairs_done)
+        line["cpu_baseline"] = {"value": tokens / (dt * scale), "unit": "tokens/s", "cores": nthreads,
+                                "kind": "oracle", "sample": f"the 2 shortest hits and the 2 shortest misses "
+                                                            f"({dt:.2f} s), extrapolated by unmasked pairs "
+                                                            f"(x{scale:.0f})"}
+    del kp, vp, ws, g
+    torch.cuda.empty_cache()
+    return line
 
 
 def cpu_oracle_layer(layer, nthreads=None):
@@ -359,6 +561,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-history sub-line")
+    ap.add_argument("--no-mixed", action="store_true", help="skip the mixed-batch sub-line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["paged", "prefill"], default=None,
                     help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
@@ -384,14 +588,19 @@ def main():
         for _ in range(args.warmup):
             cpu_oracle_layer(layer, nthreads)
         times = [cpu_oracle_layer(layer, nthreads) for _ in range(args.steps)]
-        t_layer = statistics.mean(times)
+        t_layer = statistics.median(times)
         value = layer.Tn / (t_layer * args.layers)
         print(json.dumps({
             "impl": "reference", "metric": METRIC, "value": value, "unit": "new tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_layer * args.layers * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_layer * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "paged cache hit x 8 layers (one layer timed per step, scaled by 8)",
-                       "global_batch": layer.B, "seq_len": int(layer.cached_lens.max()), "parallelism": "none"},
+            "config": {"workload": "paged cache hit x 8 layers: 8 users, cached U[1024,4096], 16 appended + 64 "
+                                   "candidates each, H=4, D=128, P=32, 65,536-page pool; per layer kv_append + "
+                                   "paged attention",
+                       "step": "one layer (layer 0) of the stack per step; ms_per_step is that layer's median time, "
+                               "value = 640 new tokens / (8 x layer time)",
+                       "layers_per_step": 1, "global_batch": layer.B, "seq_len": int(layer.cached_lens.max()),
+                       "parallelism": "none"},
             "cpu_baseline": {"value": value, "unit": "new tokens/s", "cores": nthreads, "kind": "oracle",
                              "sample": "layer 0 of the 8-layer stack: append + paged attention of all 640 new "
                                        "tokens; new tokens/s of the stack = 640 / (8 x layer time)"},
@@ -568,19 +777,25 @@ def main():
             assert torch.equal(hdst.view(torch.int16), te["out"].cpu().view(torch.int16))
             assert torch.equal(te["out"].view(torch.int16), t["out"].view(torch.int16))
 
-    prefill = None
+    prefill = long_history = mixed = None
     if rank == 0 and not args.no_prefill:
         prefill = bench_prefill(hb, device, max(5, args.steps // 2), 3, peaks)
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if rank == 0 and not args.no_long:
+        long_history = bench_long_history(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
+    if rank == 0 and not args.no_mixed:
+        mixed = bench_mixed(hb, device, max(3, args.steps // 4), 3, peaks, with_cpu)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
 
         nthreads = oracle.default_threads()
-        t_layer = cpu_oracle_layer(layers[0], nthreads)
+        samples = [cpu_oracle_layer(layers[0], nthreads) for _ in range(3)]
+        t_layer = statistics.median(samples)
         cpu = {"value": tokens / (t_layer * len(layers)), "unit": "new tokens/s", "cores": nthreads, "kind": "oracle",
-               "sample": "layer 0 of the 8-layer stack (append + paged attention of all 640 new tokens), "
-                         f"{t_layer:.2f} s; scaled as 640 / (8 x layer time)"}
+               "sample": "layer 0 of the 8-layer stack (append + paged attention of all 640 new tokens), median of "
+                         f"3 runs ({', '.join(f'{x:.2f}' for x in samples)} s); scaled as 640 / (8 x layer time)"}
 
     if world > 1:
         graph.reset() if hasattr(graph, "reset") else None
@@ -626,6 +841,8 @@ def main():
         "gpu_launches": 3 * len(L),
         "clocks": clocks,
         "prefill": prefill,
+        "long_history": long_history,
+        "mixed": mixed,
     }
     print(json.dumps(line))
 

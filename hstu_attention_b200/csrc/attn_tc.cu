@@ -204,10 +204,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         pdl_launch_dependents();
         return;
     }
-    if (qrow0 >= g.N) {
-        pdl_launch_dependents();
+    if (qrow0 >= g.N)
         return;                                               // no queries here (uniform)
-    }
 
     const int32_t i0 = qrow0;                                 // position of row 0
     const int32_t last_q = min(g.N, qrow0 + kTile) - 1;
