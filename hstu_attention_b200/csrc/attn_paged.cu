@@ -33,10 +33,11 @@
 //   warp 3 lane 0   TMA producer of the V tiles (2-stage ring)
 //   warp 1          allocates TMEM; lane 0 issues S(t+2) = Q K_{t+2}^T into S buffer t%2,
 //                   then O += P_t V_t
-//   warp 2          bias producer: per tile the 255 values rab[h][bucket(d)]/2 the tile needs,
-//                   four copies shifted by one float (16-byte reads for every thread)
-//   warps 4-11      pointwise, warpgroup t%2 on tile t: warp w reads TMEM lanes (= queries)
-//                   32(w%4).. and the tile's 128 key columns in four batches; x/2 = S/2 + rab/2,
+//   warp 2          page-id staging in the prologue only
+//   warps 4-11      pointwise, warpgroup t%2 on tile t: it first writes the tile's 255 bias
+//                   values rab[h][bucket(d)]/2 (four copies shifted by one float, so every thread
+//                   reads 16-byte vectors), then warp w reads TMEM lanes (= queries) 32(w%4).. and
+//                   the tile's 128 key columns in four batches; x/2 = S/2 + rab/2,
 //                   mask, SiLU = x/2 (1 + tanh(x/2)), bf16 P into TMEM buffer t%2; warps whose
 //                   32 lanes hold no query of the group skip the arithmetic.  Epilogue:
 //                   O / n_max -> padded fp32 tile in the rings -> 512-byte rows of the plane.
@@ -72,11 +73,11 @@ constexpr uint32_t kWinStride = 264;
 constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
 constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kRingBytes = (kKStages + kVStages) * kTileBytes;
-constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
+constexpr uint32_t kOffBounds = kOffWin + 4 * kWinBuf;    // two windows per warpgroup
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffPages = kOffRab + kMaxNB * 4;
 constexpr uint32_t kOffBar = kOffPages + kMaxPageIds * 4;
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1 + 2 + 2;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;
@@ -287,17 +288,18 @@ __device__ __forceinline__ Tile tile_of(const PieceTiles& pt, int t, int32_t C)
     return g;
 }
 
-// bucket(d) for eight distances: the largest k with bounds[k] <= d (bounds[0] = 0,
-// bounds[nb] = INT_MAX).  Branchless binary search, eight searches interleaved.
-__device__ __forceinline__ void bucket_search8(const int32_t* bounds, int nb, int top, const int32_t (&d)[8],
-                                               int (&k)[8])
+// bucket(d) for kN distances: the largest k with bounds[k] <= d (bounds[0] = 0,
+// bounds[nb] = INT_MAX).  Branchless binary search, the kN searches interleaved.
+template <int kN>
+__device__ __forceinline__ void bucket_search(const int32_t* bounds, int nb, int top, const int32_t (&d)[kN],
+                                              int (&k)[kN])
 {
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < kN; ++e)
         k[e] = 0;
     for (int step = top; step > 0; step >>= 1) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < kN; ++e)
             k[e] += (bounds[min(k[e] + step, nb)] <= d[e]) ? step : 0;
     }
 }
@@ -403,8 +405,6 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t* p_full = s_empty + 2;             // [2]: P of tile t in TMEM buffer t%2
     uint64_t* p_empty = p_full + 2;             // [2]: P V of the buffer's last tile completed
     uint64_t* o_full = p_empty + 2;
-    uint64_t* win_full = o_full + 1;            // [2]
-    uint64_t* win_empty = win_full + 2;         // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* win = reinterpret_cast<float*>(smem + kOffWin);
@@ -434,8 +434,6 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_init(&s_empty[s], 128);
                 mbar_init(&p_full[s], 128);
                 mbar_init(&p_empty[s], 1);
-                mbar_init(&win_full[s], 32);
-                mbar_init(&win_empty[s], 128);
             }
             mbar_init(o_full, 1);
             *abort_flag = 0;
@@ -657,59 +655,22 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         umma_commit(o_full);
         volatile int never = 0;
         mbar_wait(o_full, 0, &never, tmo);
-    } else if (warp == 2) {
-        // ============================================================ bias window producer
-        for (int k = lane; k < a.NB; k += 32)
+    } else if (warp >= 4) {
+        // ============================================================ pointwise + epilogue
+        // rab[h]/2 and the bucket bounds (from the host, or evaluated here for many buckets)
+        const int pt_id = threadIdx.x - 128;
+        for (int k = pt_id; k < a.NB; k += 256)
             s_rab[k] = 0.5f * a.rab[(int64_t)p.h * a.NB + k];
-        if (bb.count > 0)
-            for (int k = lane; k <= a.NB; k += 32)
-                s_bounds[k] = bb.v[k];
-        else
-            named_barrier_sync(2, 32 + 256);
-        __syncwarp();
+        for (int k = pt_id; k <= a.NB; k += 256)
+            s_bounds[k] = bb.count > 0 ? bb.v[k]
+                                       : (k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound_dev(k, a.ln_nmax, a.NB)));
+        named_barrier_sync(2, 256);
         const int nb = a.NB;
         int top = 1;
         while (top * 2 <= nb)
             top *= 2;
-        bool ok = true;
-        for (int t = 0; t < n; ++t) {
-            const int wb = t & 1;
-            if (t >= 2) {
-                ok = ok && mbar_wait_warp(&win_empty[wb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
-                if (!ok)
-                    break;
-            }
-            const Tile tg = tile_of(pt, t, p.C);
-            // window index y <-> distance d = (i0 - j0 + 127) - y: query row r and key column c
-            // meet at y = 127 - r + c
-            const int32_t dist0 = i0 - tg.j0 + (kKeys - 1);
-            float* wbuf = win + wb * (kWinBuf / 4);
-            int32_t d[8];
-            int k[8];
-#pragma unroll
-            for (int yy = 0; yy < 8; ++yy)
-                d[yy] = dist0 - (lane + 32 * yy);
-            bucket_search8(s_bounds, nb, top, d, k);
-#pragma unroll
-            for (int yy = 0; yy < 8; ++yy) {
-                const int y = lane + 32 * yy;
-                const float r = s_rab[k[yy]];
-                const float val = ((y <= 2 * kKeys - 2) & (d[yy] >= 0)) ? r : 0.f;
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    wbuf[s * kWinStride + kWinPad + (y - s)] = val;
-            }
-            mbar_arrive(&win_full[wb]);
-        }
-    } else if (warp >= 4) {
-        // ============================================================ pointwise + epilogue
-        if (bb.count == 0) {
-            const int pt_id = threadIdx.x - 128;
-            for (int k = pt_id; k <= a.NB; k += 256)
-                s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound_dev(k, a.ln_nmax, a.NB));
-            named_barrier_sync(2, 32 + 256);
-        }
         const int wg = (warp - 4) >> 2;                   // this warpgroup owns tiles wg, wg + 2, ...
+        const int wt = threadIdx.x - 128 - 128 * wg;      // 0..127 within the warpgroup
         const int q0 = (warp & 3) << 5;                   // first query row (= TMEM lane) of this warp
         const int r = q0 + lane;
         const uint32_t lane_base = (uint32_t)q0 << 16;
@@ -724,10 +685,34 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int t = wg; t < n; t += 2) {
             const int sb = t & 1;                         // == wg
             const Tile tg = tile_of(pt, t, p.C);
+            // the tile's bias window, built by the warpgroup itself (two of the 255 values per
+            // thread): window index y <-> distance d = (i0 - j0 + 127) - y, so query row r and key
+            // column c meet at y = 127 - r + c.  Copy s holds the window shifted by s floats after a
+            // 4-float pad, so every reader gets 16-byte aligned vectors.  Two buffers per warpgroup:
+            // the barrier below also orders this write after every read of the buffer two tiles ago.
+            float* wbuf = win + (2 * wg + ((t >> 1) & 1)) * (kWinBuf / 4);
+            {
+                const int32_t dist0 = i0 - tg.j0 + (kKeys - 1);
+                int32_t d[2];
+                int k[2];
+                d[0] = dist0 - wt;
+                d[1] = dist0 - (wt + 128);
+                bucket_search<2>(s_bounds, nb, top, d, k);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int y = wt + 128 * e;
+                    const float val = ((y <= 2 * kKeys - 2) & (d[e] >= 0)) ? s_rab[k[e]] : 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        wbuf[c * kWinStride + kWinPad + (y - c)] = val;
+                }
+            }
+            // every warp of the warpgroup takes this barrier once per tile, also after a timed-out
+            // wait (the rest of the iteration is then skipped, never left early)
+            named_barrier_sync(4 + wg, 128);
             ok = ok && mbar_wait_warp(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
-            ok = ok && mbar_wait_warp(&win_full[sb], (t >> 1) & 1, abort_flag, tmo);
             if (!ok)
-                break;
+                continue;
             tc_fence_after();
             const int32_t kvend = tg.j0 + tg.nvalid;
             const bool full = tg.cached && tg.nvalid == kKeys;
@@ -735,12 +720,12 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int32_t diag = (row_valid && !tg.cached) ? i_abs : -1;
             const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0);
             const uint32_t pcol = tmem + lane_base + (sb ? kColP1 : kColP0);
-            const float4* wv = reinterpret_cast<const float4*>(win + sb * (kWinBuf / 4) + woff);
+            const float4* wv = reinterpret_cast<const float4*>(wbuf + woff);
             // P buffer sb is free once P V of tile t - 2 completed
             if (t >= 2) {
                 ok = ok && mbar_wait_warp(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
                 if (!ok)
-                    break;
+                    continue;
             }
             if (warp_active) {
 #pragma unroll 1
@@ -762,7 +747,6 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             } else {
                 mbar_arrive(&s_empty[sb]);               // no query rows here: nothing to compute
             }
-            mbar_arrive(&win_empty[sb]);
             if (tg.nvalid < kKeys) {
                 // V rows past the user's keys may hold anything (page tails, stale tiles):
                 // zero them so that 0 * NaN cannot reach O
@@ -772,7 +756,7 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     uint8_t* vt = smem + kOffV + vst * kTileBytes;
                     const int first = tg.nvalid > 0 ? tg.nvalid : 0;
                     const int nchunks = (kKeys - first) * 16;
-                    for (int x = (threadIdx.x - 128 - 128 * wg); x < nchunks; x += 128) {
+                    for (int x = wt; x < nchunks; x += 128) {
                         const int row = first + (x >> 4), hf = (x >> 3) & 1, ch = x & 7;
                         *reinterpret_cast<uint4*>(vt + hf * kHalf + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
                     }
