@@ -18,10 +18,12 @@
 //   warp 1      allocates all 512 TMEM columns; lane 0 issues every MMA:
 //               S_t = Q K_t^T into S buffer t%2, then O += P_{t-1} V_{t-1}, so the pointwise
 //               work on S_t overlaps the P V product of the previous tile.
-//   warp 2      bias producer: for every tile it writes the 255 distinct values
-//               rab[h][bucket(i-j)] / 2 the tile needs into a double-buffered window, in four
-//               copies shifted by one float so each pointwise thread reads 16-byte vectors.
-//   warps 4-11  two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
+//   warp 2      idle after the set-up
+//   warps 4-11  for every tile they first write the 255 distinct values rab[h][bucket(i-j)]/2
+//               the tile needs (one per thread) into a double-buffered window, in four copies
+//               shifted by one float so each thread reads 16-byte vectors; a single producer
+//               warp sharing an SM sub-partition with pointwise warps paced the whole pipeline.
+//               Two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
 //               warp w%4 owns TMEM lanes (= query rows) [32(w%4), +32).  They load S from
 //               TMEM, form x/2 = S/2 + rab/2 with packed fp32x2 FMAs, mask, compute
 //               SiLU(x) = x/2 * (1 + tanh(x/2)), and store it as bf16 P into TMEM (P buffer
@@ -64,7 +66,7 @@ constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffBar = kOffRab + kMaxNB * 4;
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1 + 2 + 2;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;     // slack to align the base to 1024
@@ -89,22 +91,22 @@ __device__ __forceinline__ TileGeo tile_geo(int32_t t, int32_t L)
     return g;
 }
 
-// bucket(d) for eight distances at once: the largest k with bounds[k] <= d, where bounds[k]
-// is the smallest distance in bucket k (bounds[0] = 0, bounds[nb] = INT_MAX, d < 0 -> 0).
-// A branchless binary search on shared memory, the eight searches interleaved so their load
-// latencies overlap.  Only integer and load instructions: the special-function pipe stays
-// free for the pointwise warps' tanh.
-__device__ __forceinline__ void bucket_search8(const int32_t* bounds, int nb, int top, const int32_t (&d)[8],
-                                               int (&k)[8])
+// bucket(d) for kN distances at once: the largest k with bounds[k] <= d, where bounds[k] is
+// the smallest distance in bucket k (bounds[0] = 0, bounds[nb] = INT_MAX, d < 0 -> 0).  A
+// branchless binary search on shared memory, the searches interleaved so their load latencies
+// overlap.  Only integer and load instructions: the special-function pipe stays free for tanh.
+template <int kN>
+__device__ __forceinline__ void bucket_search(const int32_t* bounds, int nb, int top, const int32_t (&d)[kN],
+                                              int (&k)[kN])
 {
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
+    for (int e = 0; e < kN; ++e)
         k[e] = 0;
     // Written without short-circuit logic: a data-dependent && / || here compiles to branches
     // that diverge across lanes and serialise the warp.
     for (int step = top; step > 0; step >>= 1) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < kN; ++e)
             k[e] += (bounds[min(k[e] + step, nb)] <= d[e]) ? step : 0;
     }
 }
@@ -228,8 +230,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* p_full = s_empty + 2;             // [2]
     uint64_t* p_empty = p_full + 2;             // [2]
     uint64_t* o_full = p_empty + 2;
-    uint64_t* win_full = o_full + 1;            // [2]
-    uint64_t* win_empty = win_full + 2;         // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* win = reinterpret_cast<float*>(smem + kOffWin);
@@ -251,8 +251,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&s_empty[s], 256);
             mbar_init(&p_full[s], 256);
             mbar_init(&p_empty[s], 1);
-            mbar_init(&win_full[s], 32);
-            mbar_init(&win_empty[s], 256);
         }
         mbar_init(o_full, 1);
         *abort_flag = 0;
@@ -367,63 +365,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         umma_commit(o_full);
         volatile int never = 0;
         mbar_wait(o_full, 0, &never, tmo);
-    } else if (warp == 2) {
-        // ============================================================ bias window producer
-        const int ht = lane;                              // 0..31
-        // stage rab[h]/2 and the bucket bounds here rather than before the CTA-wide barrier:
-        // the bounds come from the parameter block, whose divergent reads are serialised, and
-        // the first window is not needed before the first S tile
-        for (int k = ht; k < a.NB; k += 32)
-            s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
-        if (bb.count > 0)
-            for (int k = ht; k <= a.NB; k += 32)
-                s_bounds[k] = bb.v[k];
-        else
-            named_barrier_sync(2, 32 + 256);          // device-evaluated bounds (warps 4-11)
-        __syncwarp();
-        const int nb = a.NB;
-        int top = 1;                                      // largest power of two <= nb
-        while (top * 2 <= nb)
-            top *= 2;
-        bool ok = true;
-        for (int t = 0; t < n; ++t) {
-            const int wb = t & 1;
-            if (t >= 2) {
-                ok = ok && mbar_wait_warp(&win_empty[wb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
-                if (!ok)
-                    break;
-            }
-            const TileGeo tg = tile_geo(t, g.L);
-            const int32_t dist0 = i0 - tg.j0 + (kTile - 1);       // distance at window index 0
-            float* wbuf = win + wb * (kWinBuf / 4);
-            int32_t d[8];
-            int k[8];
-#pragma unroll
-            for (int yy = 0; yy < 8; ++yy)
-                d[yy] = dist0 - (ht + 32 * yy);
-            bucket_search8(s_bounds, nb, top, d, k);
-#pragma unroll
-            for (int yy = 0; yy < 8; ++yy) {
-                const int y = ht + 32 * yy;
-                const float r = s_rab[k[yy]];
-                const float val = ((y <= 2 * kTile - 2) & (d[yy] >= 0)) ? r : 0.f;
-                // copy s holds the window shifted by s floats after a 4-float pad, so every
-                // lane stores all four copies without a branch
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    wbuf[s * kWinStride + kWinPad + (y - s)] = val;
-            }
-            mbar_arrive(&win_full[wb]);
-        }
     } else if (warp >= 4) {
         // ============================================================ pointwise + epilogue
         const int pt = threadIdx.x - 128;                 // 0..255
-        if (bb.count == 0) {
-            // bounds not passed by the host (many buckets): evaluate them for the bias warp
-            for (int k = pt; k <= a.NB; k += 256)
-                s_bounds[k] = k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB));
-            named_barrier_sync(2, 32 + 256);
-        }
+        // rab[h]/2 and the bucket bounds (from the host, or evaluated here for many buckets)
+        for (int k = pt; k < a.NB; k += 256)
+            s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
+        for (int k = pt; k <= a.NB; k += 256)
+            s_bounds[k] = bb.count > 0 ? bb.v[k]
+                                       : (k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB)));
+        named_barrier_sync(2, 256);
+        const int nb = a.NB;
+        int top = 1;
+        while (top * 2 <= nb)
+            top *= 2;
         const int wg = (warp - 4) >> 2;                   // key-column half
         const int r = ((warp & 3) << 5) + lane;           // query row in the block (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -440,12 +395,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int vst = t % kVStages;
             const int sb = t & 1;
             const TileGeo tg = tile_geo(t, g.L);
+            // the tile's bias window, one of its 255 values per pointwise thread: window index y <->
+            // distance d = (i0 - j0 + 127) - y, so query row r and key column c meet at y =
+            // 127 - r + c; copy s holds the window shifted by s floats after a 4-float pad, so every
+            // reader gets 16-byte aligned vectors.  Two buffers: the barrier below also orders this
+            // write after every read of the buffer two tiles ago.
+            float* wbuf = win + sb * (kWinBuf / 4);
+            {
+                int32_t d[1] = {i0 - tg.j0 + (kTile - 1) - pt};
+                int k[1];
+                bucket_search<1>(s_bounds, nb, top, d, k);
+                const float val = ((pt <= 2 * kTile - 2) & (d[0] >= 0)) ? s_rab[k[0]] : 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    wbuf[c * kWinStride + kWinPad + (pt - c)] = val;
+            }
+            // all eight pointwise warps take this barrier once per tile, also after a timed-out
+            // wait (the rest of the iteration is then skipped, never left early)
+            named_barrier_sync(4, 256);
             ok = ok && mbar_wait_warp(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
-            ok = ok && mbar_wait_warp(&win_full[sb], (t >> 1) & 1, abort_flag, tmo);
             if (!ok)
-                break;
+                continue;
             tc_fence_after();
-            const float4* wv = reinterpret_cast<const float4*>(win + sb * (kWinBuf / 4) + woff);
+            const float4* wv = reinterpret_cast<const float4*>(wbuf + woff);
             const bool full = (qrow0 + kTile - 1 < g.N) && (tg.j0 + kTile - 1 < tg.kvend) &&
                               (tg.j0 + kTile - 1 <= i0) && (tg.j0 + kTile - 1 < g.hist);
             const int32_t lim = min(lim_row, tg.kvend);
@@ -469,12 +441,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 silu_cols32<false>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag);
             else
                 silu_cols32<true>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag);
-            mbar_arrive(&win_empty[sb]);
             // P buffer sb is free once P V of tile t - 2 completed
             if (t >= 2) {
                 ok = ok && mbar_wait_warp(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
                 if (!ok)
-                    break;
+                    continue;
             }
             tmem_st_32x32b_x32(tmem + lane_base + (sb ? kColP1 : kColP0) + wg * 32,
                                *reinterpret_cast<const uint32_t(*)[32]>(&packed[0]));
