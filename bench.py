@@ -39,10 +39,14 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 # batch, from one `ncu --set full` capture of the attention and LayerNorm kernels (ncu flushes
 # caches, so the LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for
 # the kernel sources they were taken from (hash below); otherwise the bench reports traffic as null.
-PAGED_TRAFFIC_BYTES = 41.923328e6 + 3.84e3 + 6.571008e6
-PAGED_TRAFFIC_SOURCES = "fb7c6ce90c26ea98"
+PAGED_TRAFFIC_BYTES = 41.911808e6 + 9.728e3 + 6.407e6
+PAGED_TRAFFIC_SOURCES = "1ac49181580a31b0"
 # the same kind of capture for the jagged prefill attention kernel
-PREFILL_TRAFFIC_BYTES = 63.268352e6 + 11.785728e6
+PREFILL_TRAFFIC_BYTES = 63.222528e6 + 11.850752e6
+# long-history attention kernel: DRAM bytes of one call on the batch's first 8 users (the capture
+# size rule), 383.65 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
+# by that ratio (traffic grows with the pages read)
+LONG_TRAFFIC_RATIO = (379.032320e6 + 4.616704e6) / 371602680
 
 
 def kernel_sources_hash() -> str:
@@ -390,7 +394,11 @@ def bench_long_history(hb, device, steps, warmup, peaks, with_cpu):
             "algorithmic_bytes_per_call": nbytes, "flops_per_call": flops,
             "roofline": {"bound": "hbm and tensor (at the ridge)", "achieved_gbs": gbs, "hbm_peak_gbs": hbm,
                          "hbm_frac": gbs / hbm, "achieved_tflops": tf, "bf16_peak_tflops": bf16,
-                         "tensor_frac": tf / bf16, "frac": max(gbs / hbm, tf / bf16)},
+                         "tensor_frac": tf / bf16, "frac": max(gbs / hbm, tf / bf16),
+                         "traffic": (LONG_TRAFFIC_RATIO * nbytes
+                                     if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None),
+                         "traffic_note": "ncu DRAM bytes of the attention kernel on the first 8 users, scaled to "
+                                         "the full call by algorithmic bytes (1.03x algorithmic)"},
             "l2": "inputs larger than L2 (1.69 GB of distinct pages per call)"}
     if with_cpu:
         import oracle
@@ -531,7 +539,6 @@ def profile_case(case, calls):
     if case == "paged":
         c = gen.config3_paged_layers(layers=1)[0]
         ck, cv, cpt = c.compact_pool()
-        import dataclasses
 
         compact = dataclasses.replace(c, num_pages=int(ck.shape[0]), page_table=cpt,
                                       page_ids=np.arange(ck.shape[0], dtype=np.int32))
@@ -540,6 +547,30 @@ def profile_case(case, calls):
         for _ in range(calls):
             hb.paged_fwd(p, t["q"], t["k"], t["v"], t["u"], kp, vp, t["pt"], t["cl"], t["nl"], t["nt"], t["rab"],
                          max_new=c.max_new, workspace=ws, out=t["out"])
+    elif case == "long":
+        # the first 8 users of the long-history batch (about 0.4 GB of pages)
+        c = gen.config4_long()
+        c = dataclasses.replace(c, cached_lens=c.cached_lens[:8], new_lens=c.new_lens[:8], num_targets=c.num_targets[:8],
+                                append_lens=c.append_lens[:8], page_table=c.page_table[:8],
+                                q_new=c.q_new[:2048], k_new=c.k_new[:2048], v_new=c.v_new[:2048], u_new=c.u_new[:2048])
+        dev = torch.device("cuda", 0)
+        p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max, page_size=c.P, num_pages=c.num_pages,
+                      max_pages_per_user=c.max_pages)
+        kp = torch.zeros((c.num_pages, c.H, c.P, c.D), dtype=torch.bfloat16, device=dev)
+        vp = torch.zeros_like(kp)
+        used = np.unique(c.page_table[c.page_table >= 0])
+        where = np.full(c.num_pages, -1, dtype=np.int64)
+        where[c.page_ids] = np.arange(c.page_ids.shape[0])
+        used = used[where[used] >= 0]
+        pos = where[used]
+        ids = torch.from_numpy(used.astype(np.int64)).to(dev)
+        kp[ids] = _to_dev(c.pool_k[pos], dev)
+        vp[ids] = _to_dev(c.pool_v[pos], dev)
+        t = [_to_dev(x, dev) for x in (c.q_new, c.k_new, c.v_new, c.u_new)]
+        meta = [_to_dev(x, dev) for x in (c.page_table, c.cached_lens, c.new_lens, c.num_targets, c.rab)]
+        ws = hb.Workspace(p, c.B, c.Tn, c.max_new)
+        for _ in range(calls):
+            hb.paged_fwd(p, *t, kp, vp, *meta, max_new=c.max_new, workspace=ws)
     else:
         c = gen.config2_prefill()
         d = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)  # noqa
@@ -564,7 +595,7 @@ def main():
     ap.add_argument("--no-long", action="store_true", help="skip the long-history sub-line")
     ap.add_argument("--no-mixed", action="store_true", help="skip the mixed-batch sub-line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["paged", "prefill"], default=None,
+    ap.add_argument("--profile-case", choices=["paged", "prefill", "long"], default=None,
                     help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
