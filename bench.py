@@ -514,6 +514,99 @@ def bench_mixed(hb, device, steps, warmup, peaks, with_cpu):
     return line
 
 
+def bench_cache_ops(hb, device, steps, warmup, peaks):
+    """Sub-line: the cache-management copies at the paged configuration's page shape (H=4, D=128,
+    P=32, bf16: 32 KB of K and 32 KB of V per page) and the host manager's prepare latency.
+      onboard -- the cached pages of layer 0's 8 users (seed 1003, 640 pages) from a pinned host
+                 pool into their scattered GPU pages, one kv_page_copy;
+      offload -- the same pages from the GPU pool back to the host pool;
+      compact -- 16,384 scattered pages moved within the 65,536-page GPU pool (disjoint sets).
+    The host-link copies are set against one contiguous cudaMemcpyAsync of the same number of
+    bytes between the same pinned buffer and device memory (the DMA engines' rate on this box);
+    the in-pool move against HBM bandwidth."""
+    import torch
+
+    layer = gen.config3_paged_layers(layers=1)[0]
+    H, D, P, G = layer.H, layer.D, layer.P, layer.num_pages
+    p = hb.params(H, D, torch.bfloat16, layer.NB, layer.n_max, page_size=P, num_pages=G,
+                  max_pages_per_user=layer.max_pages)
+    ws = hb.Workspace(p, 1, 1, 1, device=device)
+    gk = torch.zeros((G, H, P, D), dtype=torch.bfloat16, device=device)
+    gv = torch.zeros_like(gk)
+    gpu_pages = np.concatenate([layer.page_table[b, :(int(layer.cached_lens[b]) + P - 1) // P]
+                                for b in range(layer.B)]).astype(np.int32)
+    n = len(gpu_pages)
+    hk = torch.zeros((n, H, P, D), dtype=torch.bfloat16).pin_memory()
+    hv = torch.zeros((n, H, P, D), dtype=torch.bfloat16).pin_memory()
+    on = torch.from_numpy(np.stack([np.arange(n, dtype=np.int32), gpu_pages], 1)).to(device)
+    off = torch.from_numpy(np.stack([gpu_pages, np.arange(n, dtype=np.int32)], 1)).to(device)
+    rng = np.random.default_rng(7)
+    perm = rng.permutation(G).astype(np.int32)
+    moves = torch.from_numpy(np.stack([perm[:16384], perm[16384:32768]], 1)).to(device)
+    page_bytes = H * P * D * 2 * 2
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms_on = timed(lambda: hb.kv_page_copy(p, hk, hv, gk, gv, on, workspace=ws), steps)
+    ms_off = timed(lambda: hb.kv_page_copy(p, gk, gv, hk, hv, off, workspace=ws), steps)
+    ms_mv = timed(lambda: hb.kv_page_copy(p, gk, gv, gk, gv, moves, workspace=ws), steps)
+    assert ws.status() == 0
+    # the DMA reference: the same bytes as one contiguous copy each way
+    dflat = torch.empty(n * page_bytes // 2, dtype=torch.bfloat16, device=device)
+    hflat = torch.cat([hk.reshape(-1), hv.reshape(-1)]).pin_memory()
+    ms_h2d = timed(lambda: dflat.copy_(hflat, non_blocking=True), steps)
+    ms_d2h = timed(lambda: hflat.copy_(dflat, non_blocking=True), steps)
+    nb = n * page_bytes
+
+    def gbs(nbytes, ms):
+        return nbytes / (ms * 1e-3) / 1e9
+
+    # the host manager: a 65,536-page GPU tier and a 16,384-page host tier kept full by misses
+    cache = hb.KVCache(G, 16384, P, 256)
+    lat = []
+    uid = 0
+    for i in range(3000):
+        ids = list(range(uid, uid + layer.B))
+        uid += layer.B
+        t0 = time.perf_counter()
+        cache.prepare(ids, [int(x) for x in rng.integers(1024, 4096, layer.B)])
+        lat.append(time.perf_counter() - t0)
+    st = cache.stats()
+    cache.close()
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    line = {"workload": "cache copies at H=4, D=128, P=32 bf16 (64 KB of K+V per page): onboard/offload of layer "
+                        f"0's {n} cached pages (seed 1003) between a pinned host pool and the 65,536-page GPU pool; "
+                        "compaction move of 16,384 scattered pages within the GPU pool",
+            "onboard": {"pages": n, "bytes": nb, "ms": ms_on, "gbs": gbs(nb, ms_on),
+                        "dma_contiguous_gbs": gbs(nb, ms_h2d), "frac_of_dma": ms_h2d / ms_on},
+            "offload": {"pages": n, "bytes": nb, "ms": ms_off, "gbs": gbs(nb, ms_off),
+                        "dma_contiguous_gbs": gbs(nb, ms_d2h), "frac_of_dma": ms_d2h / ms_off},
+            "compact": {"pages": 16384, "bytes_moved": 16384 * page_bytes, "ms": ms_mv,
+                        "roofline": {"bound": "hbm", "achieved": gbs(2 * 16384 * page_bytes, ms_mv), "peak": hbm,
+                                     "unit": "GB/s", "frac": gbs(2 * 16384 * page_bytes, ms_mv) / hbm,
+                                     "note": "read + write bytes"}},
+            "prepare": {"calls": len(lat), "batch": layer.B, "median_us": statistics.median(lat) * 1e6,
+                        "p99_us": float(np.percentile(lat, 99)) * 1e6,
+                        "pool": "65,536 GPU pages + 16,384 host pages, every batch 8 new users of U[1024,4096) "
+                                "tokens, so each call evicts and offloads (the host tier drops the oldest)",
+                        "final_stats": st},
+            "launches": 3}
+    del gk, gv, hk, hv, dflat, hflat
+    torch.cuda.empty_cache()
+    return line
+
+
 def cpu_oracle_layer(layer, nthreads=None):
     """Oracle time for one layer (append + paged attention of all new tokens)."""
     import oracle
@@ -594,6 +687,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-history sub-line")
     ap.add_argument("--no-mixed", action="store_true", help="skip the mixed-batch sub-line")
+    ap.add_argument("--no-cache-ops", action="store_true", help="skip the cache-management sub-line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["paged", "prefill", "long"], default=None,
                     help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
@@ -808,7 +902,7 @@ def main():
             assert torch.equal(hdst.view(torch.int16), te["out"].cpu().view(torch.int16))
             assert torch.equal(te["out"].view(torch.int16), t["out"].view(torch.int16))
 
-    prefill = long_history = mixed = None
+    prefill = long_history = mixed = cache_ops = None
     if rank == 0 and not args.no_prefill:
         prefill = bench_prefill(hb, device, max(5, args.steps // 2), 3, peaks)
     with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -816,6 +910,8 @@ def main():
         long_history = bench_long_history(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
     if rank == 0 and not args.no_mixed:
         mixed = bench_mixed(hb, device, max(3, args.steps // 4), 3, peaks, with_cpu)
+    if rank == 0 and not args.no_cache_ops:
+        cache_ops = bench_cache_ops(hb, device, max(5, args.steps // 2), 3, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -874,6 +970,7 @@ def main():
         "prefill": prefill,
         "long_history": long_history,
         "mixed": mixed,
+        "cache_ops": cache_ops,
     }
     print(json.dumps(line))
 

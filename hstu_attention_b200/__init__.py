@@ -31,6 +31,12 @@ DEV_BAD_NMAX = 1 << 2
 DEV_TIMEOUT = 1 << 3
 
 ERR_SCRATCH_LIMIT = -5
+ERR_CACHE_FULL = -6
+ERR_OUTPUT_CAPACITY = -7
+
+TIER_MISS = 0
+TIER_GPU = 1
+TIER_HOST = 2
 
 FLAG_OVERLAP_PREVIOUS = 1 << 0
 
@@ -47,6 +53,15 @@ EXPORTED = (
     "hstu_attn_paged_fwd_noalloc",
     "hstu_kv_append",
     "hstu_bucket_table",
+    "hstu_cache_create",
+    "hstu_cache_destroy",
+    "hstu_cache_lookup",
+    "hstu_cache_prepare",
+    "hstu_cache_evict",
+    "hstu_cache_compact",
+    "hstu_cache_page_rows",
+    "hstu_cache_stats",
+    "hstu_kv_page_copy",
 )
 
 
@@ -109,6 +124,24 @@ def load(path: Optional[str] = None):
             lib.hstu_kv_append.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, vp, sz, vp]
             lib.hstu_bucket_table.restype = ctypes.c_int
             lib.hstu_bucket_table.argtypes = [pp, i32, vp, vp]
+            lib.hstu_cache_create.restype = ctypes.c_int
+            lib.hstu_cache_create.argtypes = [i32, i32, i32, i32, ctypes.POINTER(vp)]
+            lib.hstu_cache_destroy.restype = None
+            lib.hstu_cache_destroy.argtypes = [vp]
+            lib.hstu_cache_lookup.restype = ctypes.c_int
+            lib.hstu_cache_lookup.argtypes = [vp, vp, i32, vp, vp]
+            lib.hstu_cache_prepare.restype = ctypes.c_int
+            lib.hstu_cache_prepare.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, vp, vp, i32, vp, vp, i32, vp]
+            lib.hstu_cache_evict.restype = ctypes.c_int
+            lib.hstu_cache_evict.argtypes = [vp, i64, vp]
+            lib.hstu_cache_compact.restype = ctypes.c_int
+            lib.hstu_cache_compact.argtypes = [vp, vp, i32, vp]
+            lib.hstu_cache_page_rows.restype = ctypes.c_int
+            lib.hstu_cache_page_rows.argtypes = [vp, vp, i32, vp]
+            lib.hstu_cache_stats.restype = ctypes.c_int
+            lib.hstu_cache_stats.argtypes = [vp, vp]
+            lib.hstu_kv_page_copy.restype = ctypes.c_int
+            lib.hstu_kv_page_copy.argtypes = [pp, vp, vp, i32, vp, vp, i32, vp, i32, vp, sz, vp]
             _lib = lib
     return _lib
 
@@ -318,3 +351,157 @@ def bucket_table(p: HstuParams, n: int, stream=None):
     out = torch.empty(int(n), dtype=torch.int32, device="cuda")
     _check(load().hstu_bucket_table(ctypes.byref(p), int(n), _ptr(out), _stream(stream)), "hstu_bucket_table")
     return out
+
+
+class CacheFull(HstuError):
+    """hstu_cache_prepare: the batch does not fit in the GPU tier even with every other user evicted."""
+
+
+class KVCache:
+    """Host-side manager of the two-tier paged KV cache (hstu_cache_* in include/hstu.h).
+
+    It owns no device memory: it hands out page ids of a GPU pool and a pinned host pool that
+    the caller allocates ([pages, H, P, D] for K and for V), and returns the page copies that
+    ``kv_page_copy`` performs.  Arrays come back as numpy int32/int64 arrays.
+    """
+
+    def __init__(self, gpu_pages: int, host_pages: int, page_size: int, max_pages_per_user: int):
+        import numpy as np  # noqa: F401  (numpy is what the results are returned in)
+
+        self.gpu_pages, self.host_pages = int(gpu_pages), int(host_pages)
+        self.page_size, self.max_pages_per_user = int(page_size), int(max_pages_per_user)
+        h = ctypes.c_void_p()
+        _check(load().hstu_cache_create(self.gpu_pages, self.host_pages, self.page_size, self.max_pages_per_user,
+                                        ctypes.byref(h)), "hstu_cache_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None) and self._h.value:
+            load().hstu_cache_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @staticmethod
+    def _ids(ids):
+        import numpy as np
+
+        return np.ascontiguousarray(np.asarray(ids, dtype=np.int64).reshape(-1))
+
+    def lookup(self, ids):
+        """(tiers, stored lengths) of the users; changes nothing."""
+        import numpy as np
+
+        ids = self._ids(ids)
+        tiers = np.zeros(len(ids), np.int32)
+        lens = np.zeros(len(ids), np.int32)
+        _check(load().hstu_cache_lookup(self._h, ids.ctypes.data, len(ids), tiers.ctypes.data, lens.ctypes.data),
+               "hstu_cache_lookup")
+        return tiers, lens
+
+    def prepare(self, ids, append_lens) -> dict:
+        """Allocate for one batch: returns tier_before, cached_lens, page_rows [B, max_pages],
+        offload [n, 2] (GPU page, host page), onboard [n, 2] (host page, GPU page), dropped ids."""
+        import numpy as np
+
+        ids = self._ids(ids)
+        app = np.ascontiguousarray(np.asarray(append_lens, dtype=np.int32).reshape(-1))
+        if len(app) != len(ids):
+            raise HstuError("one append length per user id")
+        B = len(ids)
+        tiers = np.zeros(B, np.int32)
+        cached = np.zeros(B, np.int32)
+        rows = np.zeros((B, self.max_pages_per_user), np.int32)
+        cap_off = cap_on = cap_drop = 64
+        while True:
+            off = np.zeros((cap_off, 2), np.int32)
+            on = np.zeros((cap_on, 2), np.int32)
+            drop = np.zeros(cap_drop, np.int64)
+            n_off, n_on, n_drop = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+            rc = load().hstu_cache_prepare(self._h, ids.ctypes.data, app.ctypes.data, B, tiers.ctypes.data,
+                                           cached.ctypes.data, rows.ctypes.data, off.ctypes.data, cap_off,
+                                           ctypes.byref(n_off), on.ctypes.data, cap_on, ctypes.byref(n_on),
+                                           drop.ctypes.data, cap_drop, ctypes.byref(n_drop))
+            if rc == ERR_OUTPUT_CAPACITY:
+                cap_off, cap_on, cap_drop = (max(cap_off, n_off.value), max(cap_on, n_on.value),
+                                             max(cap_drop, n_drop.value))
+                continue
+            if rc == ERR_CACHE_FULL:
+                raise CacheFull(load().hstu_error_string(rc).decode())
+            _check(rc, "hstu_cache_prepare")
+            return {"tier_before": tiers, "cached_lens": cached, "page_rows": rows,
+                    "offload": off[:n_off.value].copy(), "onboard": on[:n_on.value].copy(),
+                    "dropped": drop[:n_drop.value].copy()}
+
+    def evict(self, uid: int) -> int:
+        tier = ctypes.c_int32()
+        _check(load().hstu_cache_evict(self._h, int(uid), ctypes.byref(tier)), "hstu_cache_evict")
+        return int(tier.value)
+
+    def compact(self):
+        """(from, to) GPU page moves [n, 2] that pack the residents into pages [0, live)."""
+        import numpy as np
+
+        moves = np.zeros((max(self.gpu_pages, 1), 2), np.int32)
+        n = ctypes.c_int32()
+        _check(load().hstu_cache_compact(self._h, moves.ctypes.data, self.gpu_pages, ctypes.byref(n)),
+               "hstu_cache_compact")
+        return moves[:n.value].copy()
+
+    def page_rows(self, ids):
+        import numpy as np
+
+        ids = self._ids(ids)
+        rows = np.zeros((len(ids), self.max_pages_per_user), np.int32)
+        _check(load().hstu_cache_page_rows(self._h, ids.ctypes.data, len(ids), rows.ctypes.data),
+               "hstu_cache_page_rows")
+        return rows
+
+    def stats(self) -> dict:
+        import numpy as np
+
+        s = np.zeros(5, np.int64)
+        _check(load().hstu_cache_stats(self._h, s.ctypes.data), "hstu_cache_stats")
+        return {"free_gpu": int(s[0]), "free_host": int(s[1]), "gpu_users": int(s[2]), "host_users": int(s[3]),
+                "clock": int(s[4])}
+
+
+def _ptr_addressable(t, name):
+    """Pointer of a CUDA tensor or of a pinned host tensor (which the device addresses directly)."""
+    if t is None:
+        raise HstuError(f"{name} is required")
+    if not t.is_contiguous():
+        raise HstuError(f"{name} must be contiguous")
+    if not t.is_cuda and not t.is_pinned():
+        raise HstuError(f"{name} must be a CUDA tensor or pinned host memory")
+    return t.data_ptr()
+
+
+def kv_page_copy(p: HstuParams, src_k, src_v, dst_k, dst_v, pairs, *, workspace: Workspace, stream=None):
+    """hstu_kv_page_copy: for each (from, to) row of ``pairs`` ([n, 2] int32, CUDA or pinned),
+    copy page ``from`` of (src_k, src_v) to page ``to`` of (dst_k, dst_v).  Pools are
+    [pages, H, P, D] CUDA tensors or pinned host tensors (onboard: host -> GPU, offload:
+    GPU -> host, compaction: within the GPU pool)."""
+    import torch
+
+    want = torch.bfloat16 if p.dtype == HSTU_DTYPE_BF16 else torch.float32
+    for name, t in (("src_k", src_k), ("src_v", src_v), ("dst_k", dst_k), ("dst_v", dst_v)):
+        if t.dtype != want or t.dim() != 4 or tuple(t.shape[1:]) != (p.num_heads, p.page_size, p.head_dim):
+            raise HstuError(f"{name} must be {want} [pages, {p.num_heads}, {p.page_size}, {p.head_dim}], "
+                            f"got {t.dtype} {tuple(t.shape)}")
+    if src_k.shape != src_v.shape or dst_k.shape != dst_v.shape:
+        raise HstuError("K and V pools must have the same shape")
+    if pairs.dtype != torch.int32 or pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise HstuError("pairs must be int32 [n, 2]")
+    n = pairs.shape[0]
+    if n == 0:
+        return
+    rc = load().hstu_kv_page_copy(ctypes.byref(p), _ptr_addressable(src_k, "src_k"), _ptr_addressable(src_v, "src_v"),
+                                  src_k.shape[0], _ptr_addressable(dst_k, "dst_k"), _ptr_addressable(dst_v, "dst_v"),
+                                  dst_k.shape[0], _ptr_addressable(pairs, "pairs"), n, workspace.ptr,
+                                  workspace.nbytes, _stream(stream))
+    _check(rc, "hstu_kv_page_copy")

@@ -3,7 +3,8 @@
     python -m hstu_attention_b200.build [--force] [--verbose-ptxas]
 
 Every .cu file under csrc/ is compiled (in parallel) with
-``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` and linked into
+``-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`` (the .cpp files, host code only, with
+the same nvcc and flags) and linked into
 ``hstu_attention_b200/libhstu_b200.so`` with the CUDA runtime linked statically, so the
 library needs only the NVIDIA driver at run time.  Object files go to ``_build/``.
 """
@@ -35,7 +36,7 @@ def nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():
@@ -57,7 +58,8 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) 
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
+        stem, ext = os.path.splitext(os.path.basename(src))
+        obj = os.path.join(BUILD, stem + ext.replace(".", "_") + ".o")
         cmd = [exe] + NVCC_FLAGS + extra + ["-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:

@@ -257,6 +257,9 @@ const char* hstu_error_string(int code)
     case HSTU_ERR_CUDA: return "CUDA error";
     case HSTU_ERR_SCRATCH_LIMIT:
         return "request needs more than the 8 MiB built-in scratch of hstu_attn_paged_fwd_noalloc";
+    case HSTU_ERR_CACHE_FULL:
+        return "the batch does not fit in the GPU tier of the KV cache even with every other user evicted";
+    case HSTU_ERR_OUTPUT_CAPACITY: return "an output array of a cache call is too small";
     default: return "unknown error";
     }
 }
@@ -331,6 +334,71 @@ int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages,
     launch_kv_append(k_pages, v_pages, page_table, k_new, v_new, cached_lens, new_lens, num_targets, B, total_new,
                      params->num_heads, params->head_dim, esize_of(params), params->page_size, params->num_pages,
                      params->max_pages_per_user, max_new, workspace, static_cast<cudaStream_t>(stream));
+    return finish(static_cast<cudaStream_t>(stream));
+}
+
+// `bytes` bytes from p are addressable by the current device: device memory of this device,
+// managed memory, or pinned host memory mapped into the device's address space.  Both ends are
+// checked and must belong to one mapping; *dev_out receives the device address of p.
+static bool device_addressable(const void* p, size_t bytes, const void** dev_out)
+{
+    int dev = -1;
+    if (!p || bytes == 0 || cudaGetDevice(&dev) != cudaSuccess)
+        return false;
+    const char* ends[2] = {static_cast<const char*>(p), static_cast<const char*>(p) + (bytes - 1)};
+    const char* base = nullptr;
+    for (int e = 0; e < 2; ++e) {
+        cudaPointerAttributes a{};
+        if (cudaPointerGetAttributes(&a, ends[e]) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+        if (a.type == cudaMemoryTypeDevice) {
+            if (a.device != dev)
+                return false;
+        } else if (a.type != cudaMemoryTypeHost && a.type != cudaMemoryTypeManaged) {
+            return false;
+        }
+        const char* dp = static_cast<const char*>(a.devicePointer);
+        if (!dp)
+            return false;
+        if (e == 0)
+            base = dp;
+        else if (dp != base + (bytes - 1))
+            return false;
+    }
+    *dev_out = base;
+    return true;
+}
+
+int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const void* src_v, int32_t src_pages,
+                      void* dst_k, void* dst_v, int32_t dst_pages, const int32_t* pairs, int32_t n_pairs,
+                      void* workspace, size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, true);
+    if (rc != HSTU_OK)
+        return rc;
+    if (n_pairs < 0 || src_pages < 0 || dst_pages < 0)
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (n_pairs == 0)
+        return HSTU_OK;
+    if (!src_k || !src_v || !dst_k || !dst_v || !pairs || src_pages == 0 || dst_pages == 0)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v))
+        return HSTU_ERR_INVALID_ARG;
+    const int64_t page_bytes =
+        (int64_t)params->num_heads * params->page_size * params->head_dim * esize_of(params);
+    const void *sk, *sv, *dk, *dv, *pr;
+    if (!device_addressable(src_k, (size_t)(page_bytes * src_pages), &sk) ||
+        !device_addressable(src_v, (size_t)(page_bytes * src_pages), &sv) ||
+        !device_addressable(dst_k, (size_t)(page_bytes * dst_pages), &dk) ||
+        !device_addressable(dst_v, (size_t)(page_bytes * dst_pages), &dv) ||
+        !device_addressable(pairs, (size_t)n_pairs * 8, &pr))
+        return HSTU_ERR_INVALID_ARG;
+    launch_kv_page_copy(sk, sv, const_cast<void*>(dk), const_cast<void*>(dv), static_cast<const int32_t*>(pr),
+                        n_pairs, src_pages, dst_pages, page_bytes, workspace, static_cast<cudaStream_t>(stream));
     return finish(static_cast<cudaStream_t>(stream));
 }
 

@@ -1,0 +1,68 @@
+// kv_pages.cu -- whole-page copies between KV pools: the onboard (pinned host pool -> GPU pool),
+// offload (GPU pool -> pinned host pool) and compaction (within the GPU pool) moves of the
+// two-tier KV cache (NVIDIA blog "Deploying an HSTU Generative Recommender with NVIDIA
+// Dynamo-Triton", section "Why serving large sequential recommenders is hard": a host tier
+// beside the paged GPU table, with onboard and offload operations).
+//
+// A page is H * P * D elements, the same contiguous block in both pools, so a copy is a
+// gather/scatter of fixed-size blocks by page id.  Grid (chunks of a page, pairs, {K, V}); a
+// thread moves kUnroll 16-byte vectors and issues all its loads before its stores, so each
+// block keeps 16 KB of reads in flight.  That covers HBM latency for the in-pool copy and the
+// much longer latency of reads from pinned host memory over the host link (the SMs address the
+// host pool directly; no staging buffer and no per-page copy call).
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hstu {
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+
+__global__ void __launch_bounds__(kCopyThreads)
+kv_page_copy_kernel(const uint4* __restrict__ src_k, const uint4* __restrict__ src_v, uint4* __restrict__ dst_k,
+                    uint4* __restrict__ dst_v, const int32_t* __restrict__ pairs, int32_t n_pairs, int32_t src_pages,
+                    int32_t dst_pages, int64_t page_vecs, void* ws)
+{
+    const uint4* src = blockIdx.z ? src_v : src_k;
+    uint4* dst = blockIdx.z ? dst_v : dst_k;
+    const int64_t first = (int64_t)blockIdx.x * (kCopyThreads * kCopyUnroll) + threadIdx.x;
+    for (int64_t i = blockIdx.y; i < n_pairs; i += gridDim.y) {
+        const int32_t s = pairs[2 * i], d = pairs[2 * i + 1];
+        if (s < 0 || s >= src_pages || d < 0 || d >= dst_pages) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0)
+                set_flag(ws, HSTU_DEV_BAD_PAGE);
+            continue;
+        }
+        const uint4* sp = src + (int64_t)s * page_vecs;
+        uint4* dp = dst + (int64_t)d * page_vecs;
+        uint4 r[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t x = first + u * kCopyThreads;
+            if (x < page_vecs)
+                r[u] = sp[x];
+        }
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t x = first + u * kCopyThreads;
+            if (x < page_vecs)
+                dp[x] = r[u];
+        }
+    }
+}
+
+void launch_kv_page_copy(const void* src_k, const void* src_v, void* dst_k, void* dst_v, const int32_t* pairs,
+                         int32_t n_pairs, int32_t src_pages, int32_t dst_pages, int64_t page_bytes, void* ws,
+                         cudaStream_t stream)
+{
+    if (n_pairs <= 0)
+        return;
+    const int64_t page_vecs = page_bytes / 16;
+    const int64_t per_block = (int64_t)kCopyThreads * kCopyUnroll;
+    dim3 grid((unsigned)((page_vecs + per_block - 1) / per_block), (unsigned)(n_pairs < 65535 ? n_pairs : 65535), 2);
+    kv_page_copy_kernel<<<grid, kCopyThreads, 0, stream>>>(
+        static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v), static_cast<uint4*>(dst_k),
+        static_cast<uint4*>(dst_v), pairs, n_pairs, src_pages, dst_pages, page_vecs, ws);
+}
+
+}  // namespace hstu

@@ -59,8 +59,11 @@ typedef enum {
     HSTU_ERR_UNSUPPORTED = -2,  /* a shape this build does not implement */
     HSTU_ERR_WORKSPACE = -3,    /* workspace too small or misaligned */
     HSTU_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed */
-    HSTU_ERR_SCRATCH_LIMIT = -5 /* hstu_attn_paged_fwd_noalloc: the request does not fit the
-                                   library's built-in 8 MiB scratch */
+    HSTU_ERR_SCRATCH_LIMIT = -5, /* hstu_attn_paged_fwd_noalloc: the request does not fit the
+                                    library's built-in 8 MiB scratch */
+    HSTU_ERR_CACHE_FULL = -6,    /* hstu_cache_prepare: the batch does not fit in the GPU tier
+                                    even with every other user evicted */
+    HSTU_ERR_OUTPUT_CAPACITY = -7 /* a caller-sized output array of a cache call is too small */
 } hstu_status_code;
 
 typedef enum { HSTU_DTYPE_BF16 = 0, HSTU_DTYPE_FP32 = 1 } hstu_dtype;
@@ -257,6 +260,128 @@ int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages,
                    const int32_t* cached_lens, const int32_t* new_lens,
                    const int32_t* num_targets, int32_t B, int64_t total_new, int32_t max_new,
                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------
+ * KV cache management around append: a two-tier paged cache (GPU pages and pinned host pages)
+ * with LRU eviction, onboard and offload, and compaction.
+ *
+ * The pages describe the serving path's cache manager (NVIDIA blog "Deploying an HSTU
+ * Generative Recommender with NVIDIA Dynamo-Triton", section "Why serving large sequential
+ * recommenders is hard"): the GPU cache is a paged KV table supporting lookup, allocate, append
+ * and evict; when GPU space runs short, old users are evicted by an LRU-like policy; host
+ * storage is a further tier; the exported path has cache-aware operations for lookup,
+ * allocate, onboard, append and offload.  The pages give no algorithm; this library's
+ * definition is:
+ *
+ *   - A user (int64 id) is resident in at most one tier, with a stored length n (tokens),
+ *     ceil(n / P) pages of that tier in logical order, and a stamp: the number of the last
+ *     hstu_cache_prepare call that had the user in its batch.
+ *   - Free pages are handed out lowest id first.
+ *   - hstu_cache_prepare(ids, append) serves one batch (distinct ids).  With n_b the stored
+ *     length (0 on a miss), user b needs ceil((n_b + append_b) / P) GPU pages (at most
+ *     max_pages_per_user).  If the free GPU pages do not cover the batch's extra pages, GPU
+ *     residents outside the batch are evicted oldest first -- ordered by (stamp, user id) --
+ *     until they do (if even evicting all of them would not, the call fails with
+ *     HSTU_ERR_CACHE_FULL).  Evicted users are offloaded to the host tier newest first; a
+ *     victim that does not fit in the free host pages takes the pages of host residents
+ *     outside the batch that are older than itself, oldest first; if even all of those would
+ *     not make room, the victim is dropped.  Then, in batch order: GPU residents get their
+ *     extra pages, host residents of the batch are onboarded into fresh GPU pages (their
+ *     host pages are freed at the end of the call), misses get fresh pages.  Each batch
+ *     user's stamp becomes the call's number and its stored length n_b + append_b: the caller
+ *     appends those tokens (hstu_kv_append, or the prefill's append on a miss) after the copies.
+ *   - hstu_cache_compact moves GPU pages so that the residents occupy pages [0, live): the
+ *     live pages at ids >= live, ascending, go to the free ids < live, ascending.
+ *
+ * The manager is host code: it owns no device memory and launches nothing.  It returns page
+ * rows and lists of (from, to) page pairs; hstu_kv_page_copy moves the pages.  For one
+ * prepare call the caller runs, on one stream and in this order: the offload copy (GPU pool ->
+ * host pool), the onboard copy (host pool -> GPU pool), then anything that writes the batch's
+ * pages or reads them (appends, attention).  Evicted and dropped users' GPU pages may be
+ * reused by the same batch, so the offload copy must run first.
+ *
+ * All cache calls take host pointers, are synchronous, and are safe to call from several
+ * threads (each cache has its own lock).  A failed call changes nothing.
+ * ------------------------------------------------------------------------------------------ */
+
+typedef struct hstu_kv_cache hstu_kv_cache;
+
+enum { HSTU_TIER_MISS = 0, HSTU_TIER_GPU = 1, HSTU_TIER_HOST = 2 };
+
+/*
+ * Create a cache of gpu_pages GPU pages and host_pages host pages (host_pages may be 0: no host
+ * tier, evicted users are dropped), page_size P >= 1 tokens per page, at most
+ * max_pages_per_user pages per user (the row length of the page rows it returns).
+ * *out receives the handle; free it with hstu_cache_destroy.
+ */
+int hstu_cache_create(int32_t gpu_pages, int32_t host_pages, int32_t page_size,
+                      int32_t max_pages_per_user, hstu_kv_cache** out);
+void hstu_cache_destroy(hstu_kv_cache* cache);
+
+/* Lookup: for n ids, tier_out[i] = HSTU_TIER_* and len_out[i] = stored length (0 on a miss).
+ * Changes nothing (stamps included). */
+int hstu_cache_lookup(hstu_kv_cache* cache, const int64_t* user_ids, int32_t n, int32_t* tier_out,
+                      int32_t* len_out);
+
+/*
+ * Allocate for one batch of B distinct users that will append append_lens[b] >= 0 tokens each
+ * (see the definition above).  Outputs (host arrays):
+ *   tier_before_out [B]       tier of each user before the call (MISS, GPU or HOST)
+ *   cached_lens_out [B]       stored length before the call (0 on a miss): the paged
+ *                             attention's cached_lens, and where the append starts
+ *   page_table_out  [B][max_pages_per_user]  the user's GPU pages, -1 past them: the page
+ *                             table of hstu_attn_paged_fwd and hstu_kv_append
+ *   offload_pairs_out [capacity][2]  (GPU page, host page) pairs, *n_offload of them
+ *   onboard_pairs_out [capacity][2]  (host page, GPU page) pairs, *n_onboard of them
+ *   dropped_out [capacity]    users that left the cache in this call (victims that did not
+ *                             fit in the host tier, host residents that made room), in
+ *                             the order they were dropped
+ * Errors: HSTU_ERR_INVALID_ARG (null pointer, B < 0, repeated id, negative append, a user
+ * needing more than max_pages_per_user pages), HSTU_ERR_CACHE_FULL, HSTU_ERR_OUTPUT_CAPACITY
+ * (an output list longer than its capacity; the counts hold the lengths needed).
+ */
+int hstu_cache_prepare(hstu_kv_cache* cache, const int64_t* user_ids, const int32_t* append_lens,
+                       int32_t B, int32_t* tier_before_out, int32_t* cached_lens_out,
+                       int32_t* page_table_out, int32_t* offload_pairs_out,
+                       int32_t offload_capacity, int32_t* n_offload, int32_t* onboard_pairs_out,
+                       int32_t onboard_capacity, int32_t* n_onboard, int64_t* dropped_out,
+                       int32_t dropped_capacity, int32_t* n_dropped);
+
+/* Evict one user from whichever tier holds it; *tier_out = that tier (MISS if none). */
+int hstu_cache_evict(hstu_kv_cache* cache, int64_t user_id, int32_t* tier_out);
+
+/* Compaction of the GPU tier: *n_moves (from, to) pairs into move_pairs_out [capacity][2]
+ * (at most gpu_pages are ever needed); sources and destinations are disjoint, so one
+ * hstu_kv_page_copy within the GPU pool performs them.  Fetch page rows again afterwards. */
+int hstu_cache_compact(hstu_kv_cache* cache, int32_t* move_pairs_out, int32_t capacity,
+                       int32_t* n_moves);
+
+/* Current GPU page rows of n users, [n][max_pages_per_user]; all -1 for a user not on the GPU. */
+int hstu_cache_page_rows(hstu_kv_cache* cache, const int64_t* user_ids, int32_t n, int32_t* rows_out);
+
+/* stats_out[5] = free GPU pages, free host pages, users on the GPU, users on the host,
+ * number of successful prepare calls. */
+int hstu_cache_stats(hstu_kv_cache* cache, int64_t* stats_out);
+
+/*
+ * Copy whole pages: for i < n_pairs, page pairs[2i] of (src_k, src_v) to page pairs[2i+1] of
+ * (dst_k, dst_v), K and V alike; a page is H * P * D elements of params->dtype.  This is the
+ * onboard (host pool -> GPU pool), offload (GPU pool -> host pool) and compaction (within the
+ * GPU pool) copy of the cache above.
+ *   src_k, src_v : [src_pages][H][P][D];  dst_k, dst_v : [dst_pages][H][P][D]
+ *   pairs        : [n_pairs][2] int32
+ * Every pointer must be device memory of the current device or pinned host memory that the
+ * device can address (allocated with cudaHostAlloc/cudaMallocHost, or registered), 16-byte
+ * aligned; the call checks both ends of each pool and of the pair array and returns
+ * HSTU_ERR_INVALID_ARG otherwise.  Destination pages must be distinct, and within one pool no
+ * page may be both a source and a destination (the pairs run in any order).  A pair with a
+ * page id out of range is skipped and sets HSTU_DEV_BAD_PAGE in the workspace's status word
+ * (the workspace is used for nothing else).  Asynchronous on stream.
+ */
+int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const void* src_v,
+                      int32_t src_pages, void* dst_k, void* dst_v, int32_t dst_pages,
+                      const int32_t* pairs, int32_t n_pairs, void* workspace,
+                      size_t workspace_bytes, void* stream);
 
 /*
  * The library's own bucket table: table_out[d] = bucket(d) for d in [0, n), computed on the

@@ -121,6 +121,31 @@ def test_flags_and_noalloc_limit_without_gpu(lib):
     assert N(ctypes.byref(_p(n_max=8192)), *misaligned_flags) == -1
 
 
+def test_page_copy_host_validation_without_gpu(lib):
+    """The page-copy entry rejects bad arguments before it touches the device; on a machine
+    without a GPU no pointer is device-addressable, so even well-formed calls are refused."""
+    p = _p()
+    fake = 1 << 20
+    C = lib.hstu_kv_page_copy
+    good = [fake, fake, 8, fake, fake, 8, fake, 4, fake, 4096, None]
+    assert C(None, *good) == -1
+    bad = list(good)
+    bad[7] = -1                                   # n_pairs < 0
+    assert C(ctypes.byref(p), *bad) == -1
+    bad = list(good)
+    bad[8] = fake + 8                             # workspace not 256-byte aligned
+    assert C(ctypes.byref(p), *bad) == -3
+    bad = list(good)
+    bad[0] = fake + 4                             # source pool not 16-byte aligned
+    assert C(ctypes.byref(p), *bad) == -1
+    zero = list(good)
+    zero[7] = 0
+    assert C(ctypes.byref(p), *zero) == 0         # nothing to copy
+    assert C(ctypes.byref(p), *good) == -1        # not addressable by any device here
+    for code in (hb.ERR_CACHE_FULL, hb.ERR_OUTPUT_CAPACITY):
+        assert lib.hstu_error_string(code).decode() != "unknown error"
+
+
 def test_backward_host_validation_without_gpu(lib):
     """The backward entry rejects bad arguments before it enqueues anything."""
     p = _p()
