@@ -688,6 +688,9 @@ def main():
     ap.add_argument("--no-long", action="store_true", help="skip the long-history sub-line")
     ap.add_argument("--no-mixed", action="store_true", help="skip the mixed-batch sub-line")
     ap.add_argument("--no-cache-ops", action="store_true", help="skip the cache-management sub-line")
+    ap.add_argument("--e2e-upload", choices=("sm", "dma"), default="dma",
+                    help="e2e uploads: a DMA cudaMemcpyAsync per layer (default) or hstu_host_copy (the SMs read "
+                         "pinned host memory; slower here because it competes with the attention kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["paged", "prefill", "long"], default=None,
                     help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
@@ -868,7 +871,10 @@ def main():
         up.wait_event(ev_fetched[si])
         with torch.cuda.stream(up):
             for li in range(len(L)):
-                dev_in[si][li].copy_(host_in[li], non_blocking=True)
+                if args.e2e_upload == "sm":
+                    hb.host_copy(dev_in[si][li], host_in[li], stream=up)
+                else:
+                    dev_in[si][li].copy_(host_in[li], non_blocking=True)
                 ev_up[si][li].record(up)
         for li, t in enumerate(L_e2e[si]):
             stream.wait_event(ev_up[si][li])
@@ -962,6 +968,8 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": job_throughput(tokens, e2e_ms, world), "unit": "new tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "upload": ("hstu_host_copy (SM copy kernel reading pinned host memory)" if args.e2e_upload == "sm"
+                           else "cudaMemcpyAsync (DMA)"),
                 "mode": "one graph per layer; each layer's inputs in one pinned buffer (one upload per layer); "
                         "uploads and downloads overlap the neighbouring layers' kernels on two copy streams; "
                         "two sets of device buffers, so a step's uploads overlap the previous step"},

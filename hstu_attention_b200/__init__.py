@@ -62,6 +62,7 @@ EXPORTED = (
     "hstu_cache_page_rows",
     "hstu_cache_stats",
     "hstu_kv_page_copy",
+    "hstu_host_copy",
 )
 
 
@@ -142,6 +143,8 @@ def load(path: Optional[str] = None):
             lib.hstu_cache_stats.argtypes = [vp, vp]
             lib.hstu_kv_page_copy.restype = ctypes.c_int
             lib.hstu_kv_page_copy.argtypes = [pp, vp, vp, i32, vp, vp, i32, vp, i32, vp, sz, vp]
+            lib.hstu_host_copy.restype = ctypes.c_int
+            lib.hstu_host_copy.argtypes = [vp, vp, sz, vp]
             _lib = lib
     return _lib
 
@@ -505,3 +508,13 @@ def kv_page_copy(p: HstuParams, src_k, src_v, dst_k, dst_v, pairs, *, workspace:
                                   dst_k.shape[0], _ptr_addressable(pairs, "pairs"), n, workspace.ptr,
                                   workspace.nbytes, _stream(stream))
     _check(rc, "hstu_kv_page_copy")
+
+
+def host_copy(dst, src, stream=None):
+    """hstu_host_copy: copy src into dst (same number of bytes; CUDA or pinned host tensors) with
+    the GPU's SMs, asynchronously on ``stream``."""
+    n = dst.numel() * dst.element_size()
+    if src.numel() * src.element_size() != n:
+        raise HstuError("host_copy: src and dst differ in size")
+    _check(load().hstu_host_copy(_ptr_addressable(dst, "dst"), _ptr_addressable(src, "src"), n, _stream(stream)),
+           "hstu_host_copy")

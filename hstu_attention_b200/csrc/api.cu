@@ -402,6 +402,23 @@ int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const v
     return finish(static_cast<cudaStream_t>(stream));
 }
 
+int hstu_host_copy(void* dst, const void* src, size_t bytes, void* stream)
+{
+    if (bytes == 0)
+        return HSTU_OK;
+    if (!dst || !src || !aligned16(dst) || !aligned16(src))
+        return HSTU_ERR_INVALID_ARG;
+    const void *d, *s;
+    if (!device_addressable(dst, bytes, &d) || !device_addressable(src, bytes, &s))
+        return HSTU_ERR_INVALID_ARG;
+    const char* dc = static_cast<const char*>(d);
+    const char* sc = static_cast<const char*>(s);
+    if (dc < sc + bytes && sc < dc + bytes)
+        return HSTU_ERR_INVALID_ARG;    // overlapping ranges
+    launch_flat_copy(const_cast<void*>(d), s, (int64_t)bytes, static_cast<cudaStream_t>(stream));
+    return finish(static_cast<cudaStream_t>(stream));
+}
+
 // The attention part of the jagged forward: O / n_max of every query row into the fp32 plane
 // `part` ([tokens][H][D]); device-detected errors go to the workspace status word.
 static int jagged_attention(const hstu_attn_params* params, const void* q, const void* k, const void* v,

@@ -66,6 +66,8 @@ void launch_kv_page_copy(const void* src_k, const void* src_v, void* dst_k, void
                          int32_t n_pairs, int32_t src_pages, int32_t dst_pages, int64_t page_bytes, void* ws,
                          cudaStream_t stream);
 
+void launch_flat_copy(void* dst, const void* src, int64_t bytes, cudaStream_t stream);
+
 void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, const void* k_new,
                       const void* v_new, const int32_t* cached_lens, const int32_t* new_lens,
                       const int32_t* num_targets, int32_t B, int64_t total_new, int32_t H, int32_t D,

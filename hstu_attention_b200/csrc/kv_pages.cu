@@ -66,3 +66,57 @@ void launch_kv_page_copy(const void* src_k, const void* src_v, void* dst_k, void
 }
 
 }  // namespace hstu
+
+namespace hstu {
+
+// A flat copy of `nvec` 16-byte vectors plus a `tail` of fewer than 16 bytes, between any two
+// buffers the device addresses (device memory, or pinned host memory read or written over the
+// host link).  Blocks stride over the buffer; a thread keeps kFlatUnroll vectors in flight, so a
+// block has 16 KB of reads outstanding -- enough for the host link's latency with a few dozen
+// blocks.  128-thread blocks with few registers fit beside a resident attention CTA on its SM.
+constexpr int kFlatThreads = 128;
+constexpr int kFlatUnroll = 8;
+
+__global__ void __launch_bounds__(kFlatThreads)
+flat_copy_kernel(uint4* __restrict__ dst, const uint4* __restrict__ src, int64_t nvec,
+                 unsigned char* __restrict__ dtail, const unsigned char* __restrict__ stail, int tail)
+{
+    const int64_t per_block = (int64_t)kFlatThreads * kFlatUnroll;
+    for (int64_t base = (int64_t)blockIdx.x * per_block + threadIdx.x; base < nvec;
+         base += (int64_t)gridDim.x * per_block) {
+        uint4 r[kFlatUnroll];
+#pragma unroll
+        for (int u = 0; u < kFlatUnroll; ++u) {
+            const int64_t x = base + u * kFlatThreads;
+            if (x < nvec)
+                r[u] = src[x];
+        }
+#pragma unroll
+        for (int u = 0; u < kFlatUnroll; ++u) {
+            const int64_t x = base + u * kFlatThreads;
+            if (x < nvec)
+                dst[x] = r[u];
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x < tail)
+        dtail[threadIdx.x] = stail[threadIdx.x];
+}
+
+void launch_flat_copy(void* dst, const void* src, int64_t bytes, cudaStream_t stream)
+{
+    if (bytes <= 0)
+        return;
+    const int64_t nvec = bytes / 16;
+    const int tail = (int)(bytes - nvec * 16);
+    const int64_t per_block = (int64_t)kFlatThreads * kFlatUnroll;
+    int64_t blocks = (nvec + per_block - 1) / per_block;
+    if (blocks > 256)
+        blocks = 256;
+    if (blocks < 1)
+        blocks = 1;
+    flat_copy_kernel<<<(unsigned)blocks, kFlatThreads, 0, stream>>>(
+        static_cast<uint4*>(dst), static_cast<const uint4*>(src), nvec, static_cast<unsigned char*>(dst) + nvec * 16,
+        static_cast<const unsigned char*>(src) + nvec * 16, tail);
+}
+
+}  // namespace hstu

@@ -384,6 +384,18 @@ int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const v
                       size_t workspace_bytes, void* stream);
 
 /*
+ * Copy `bytes` bytes from src to dst with the GPU's SMs, as one kernel on `stream`: the upload of
+ * a call's inputs from pinned host memory (or the download of its outputs) done by the device
+ * reading and writing host memory over the host link, instead of a DMA copy.  Either pointer
+ * may be device memory of the current device or pinned host memory the device addresses
+ * (cudaHostAlloc/cudaMallocHost or registered); both 16-byte aligned; the ranges must not
+ * overlap.  Both ends of both ranges are checked before the launch (HSTU_ERR_INVALID_ARG
+ * otherwise).  Asynchronous; the caller keeps the host buffer alive and unchanged until the
+ * stream has passed the copy.  A transport choice of this library (the pages describe none).
+ */
+int hstu_host_copy(void* dst, const void* src, size_t bytes, void* stream);
+
+/*
  * The library's own bucket table: table_out[d] = bucket(d) for d in [0, n), computed on the
  * device in double precision (the function that the attention kernels use).  table_out is
  * a device int32 array of n entries.  Exposed so that tests can compare it with an

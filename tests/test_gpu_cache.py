@@ -249,3 +249,22 @@ def test_serving_loop_through_the_cache(hb):
 def test_serving_loop_without_a_host_tier(hb):
     stats = _serving_loop(hb, seed=22, steps=25, G=56, Hp=0, compact_every=0, evict_every=0)
     assert stats["dropped"] > 0 and stats["host"] == 0
+
+
+@pytest.mark.parametrize("nbytes", [16, 4096 + 7, 3 * 1024 * 1024 + 48, 41 * 1024 * 1024 + 5])
+def test_host_copy_bit_exact(hb, nbytes):
+    """hstu_host_copy moves pinned host bytes to the device and back, bit for bit, tails included."""
+    import torch
+
+    rng = np.random.default_rng(nbytes)
+    src = torch.from_numpy(rng.integers(0, 256, nbytes, dtype=np.uint8)).pin_memory()
+    mid = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    back = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
+    hb.host_copy(mid, src)
+    hb.host_copy(back, mid)
+    torch.cuda.synchronize()
+    assert torch.equal(mid.cpu(), src) and torch.equal(back, src)
+    with pytest.raises(hb.HstuError):
+        hb.host_copy(mid[:16], torch.zeros(16, dtype=torch.uint8))   # pageable host memory
+    with pytest.raises(hb.HstuError):
+        hb.host_copy(mid[16:32], mid[8:24])                           # overlapping ranges (and misaligned)
