@@ -485,8 +485,9 @@ def bench_mixed(hb, device, steps, warmup, peaks, with_cpu):
         # seeded subset: the two shortest hits (paged oracle) and the two shortest misses (prefill
         # oracle), extrapolated to the whole step by unmasked pairs
         nthreads = oracle.default_threads()
-        hsel = np.argsort(hits.cached_lens, kind="stable")[:2]
-        msel = np.argsort(misses.lengths, kind="stable")[:2]
+        # the 3 hits and 3 misses closest to the median length: a representative sample of a few s
+        hsel = np.argsort(np.abs(hits.cached_lens - np.median(hits.cached_lens)), kind="stable")[:3]
+        msel = np.argsort(np.abs(misses.lengths - np.median(misses.lengths)), kind="stable")[:3]
         t0 = time.perf_counter()
         pairs_done = 0
         for b in hsel:
@@ -506,7 +507,7 @@ def bench_mixed(hb, device, steps, warmup, peaks, with_cpu):
         dt = time.perf_counter() - t0
         scale = (hit_flops + miss_flops) / (4 * hits.D) / max(1, pairs_done)
         line["cpu_baseline"] = {"value": tokens / (dt * scale), "unit": "tokens/s", "cores": nthreads,
-                                "kind": "oracle", "sample": f"the 2 shortest hits and the 2 shortest misses "
+                                "kind": "oracle", "sample": f"the 3 hits and 3 misses nearest the median length "
                                                             f"({dt:.2f} s), extrapolated by unmasked pairs "
                                                             f"(x{scale:.0f})"}
     del kp, vp, ws, g

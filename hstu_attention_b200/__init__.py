@@ -40,6 +40,8 @@ TIER_HOST = 2
 
 FLAG_OVERLAP_PREVIOUS = 1 << 0
 
+INJECT_STALL_V = 1
+
 EXPORTED = (
     "hstu_version",
     "hstu_error_string",
@@ -63,6 +65,7 @@ EXPORTED = (
     "hstu_cache_stats",
     "hstu_kv_page_copy",
     "hstu_host_copy",
+    "hstu_test_inject",
 )
 
 
@@ -145,6 +148,8 @@ def load(path: Optional[str] = None):
             lib.hstu_kv_page_copy.argtypes = [pp, vp, vp, i32, vp, vp, i32, vp, i32, vp, sz, vp]
             lib.hstu_host_copy.restype = ctypes.c_int
             lib.hstu_host_copy.argtypes = [vp, vp, sz, vp]
+            lib.hstu_test_inject.restype = ctypes.c_int
+            lib.hstu_test_inject.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
             _lib = lib
     return _lib
 
@@ -518,3 +523,9 @@ def host_copy(dst, src, stream=None):
         raise HstuError("host_copy: src and dst differ in size")
     _check(load().hstu_host_copy(_ptr_addressable(dst, "dst"), _ptr_addressable(src, "src"), n, _stream(stream)),
            "hstu_host_copy")
+
+
+def test_inject(kind: int, wait_limit_ns: int = 0):
+    """hstu_test_inject: test-only fault injection of the time-out path (INJECT_STALL_V: the V
+    producer issues nothing and role waits give up after wait_limit_ns); kind 0 restores normal calls."""
+    _check(load().hstu_test_inject(int(kind), int(wait_limit_ns)), "hstu_test_inject")

@@ -206,6 +206,19 @@ static int finish(cudaStream_t)
 
 static constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s per in-kernel wait
 
+// Test-only fault injection (hstu_test_inject): an injected kind and the role-wait limit the
+// tensor-core kernels then use; the waits for a CTA's own copies and products keep 2 s.
+static std::atomic<uint32_t> g_inject_kind{0};
+static std::atomic<uint64_t> g_inject_limit_ns{0};
+
+static void set_waits(TcArgs& a)
+{
+    const uint32_t kind = g_inject_kind.load(std::memory_order_relaxed);
+    a.inject = kind;
+    a.timeout_ns = kind ? g_inject_limit_ns.load(std::memory_order_relaxed) : kTimeoutNs;
+    a.drain_ns = kTimeoutNs;
+}
+
 // Scratch of hstu_attn_paged_fwd_noalloc: a fixed array in the library's own device image, so
 // that callers which cannot hand over a workspace still get a paged forward.  Layout is the
 // workspace layout (status block, split counts, fp32 partial planes).  Every call on a device
@@ -402,6 +415,17 @@ int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const v
     return finish(static_cast<cudaStream_t>(stream));
 }
 
+int hstu_test_inject(uint32_t kind, uint64_t wait_limit_ns)
+{
+    if (kind & ~(uint32_t)HSTU_INJECT_STALL_V)
+        return HSTU_ERR_INVALID_ARG;
+    if (kind && (wait_limit_ns < 1000000ull || wait_limit_ns > kTimeoutNs))
+        return HSTU_ERR_INVALID_ARG;
+    g_inject_limit_ns.store(wait_limit_ns, std::memory_order_relaxed);
+    g_inject_kind.store(kind == HSTU_INJECT_STALL_V ? kInjectStallV : 0u, std::memory_order_relaxed);
+    return HSTU_OK;
+}
+
 int hstu_host_copy(void* dst, const void* src, size_t bytes, void* stream)
 {
     if (bytes == 0)
@@ -456,8 +480,8 @@ static int jagged_attention(const hstu_attn_params* params, const void* q, const
         a.qblocks = (max_seqlen + 127) / 128;
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
-        a.timeout_ns = kTimeoutNs;
         a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+        set_waits(a);
         launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), B, s);
     } else {
         SimtArgs a{};
@@ -652,8 +676,8 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.qblocks = (max_new + 127) / 128;
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
-        a.timeout_ns = kTimeoutNs;
         a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+        set_waits(a);
         launch_attn_paged(m, a, host_bounds(params->n_max, params->num_buckets), num_sms(), s);
     } else {
         SimtArgs a{};

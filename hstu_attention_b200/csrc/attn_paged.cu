@@ -509,6 +509,7 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     const bool bad_page_staged = *reinterpret_cast<volatile unsigned int*>(smem + kOffMisc + 8) != 0;
     const uint64_t tmo = a.timeout_ns;
+    const uint64_t drain = a.drain_ns;
     if ((warp == 0 || warp == 3) && lane == 0) {
         // start streaming the first tiles from HBM while the previous kernel finishes
         const bool is_v = warp == 3;
@@ -541,7 +542,8 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tma_load_3d(&tm_q, sbase + kOffQ + hf * kHalf, q_full, hf * 64, p.h, (int32_t)(p.off + qrow0));
         }
         int issued = 0;
-        for (int t = 0; t < n; ++t) {
+        const int n_issue = (is_v && (a.inject & kInjectStallV)) ? 0 : n;
+        for (int t = 0; t < n_issue; ++t) {
             const Tile tg = tile_of(pt, t, p.C);
             const int st = t % stages;
             if (t + kPrefetchTiles < n)
@@ -588,9 +590,9 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // raises the CTA-wide abort)
         volatile int never = 0;
         if (!is_v)
-            mbar_wait(q_full, 0, &never, tmo);
+            mbar_wait(q_full, 0, &never, drain);
         for (int t = (issued > stages ? issued - stages : 0); t < issued; ++t)
-            mbar_wait(&full[t % stages], (t / stages) & 1, &never, tmo);
+            mbar_wait(&full[t % stages], (t / stages) & 1, &never, drain);
     } else if (warp == 1 && lane == 0) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
@@ -654,7 +656,7 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // so tensor memory is idle before it is released)
         umma_commit(o_full);
         volatile int never = 0;
-        mbar_wait(o_full, 0, &never, tmo);
+        mbar_wait(o_full, 0, &never, drain);
     } else if (warp >= 4) {
         // ============================================================ pointwise + epilogue
         // rab[h]/2 and the bucket bounds (from the host, or evaluated here for many buckets)

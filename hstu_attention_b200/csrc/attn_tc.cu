@@ -265,6 +265,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = a.timeout_ns;
+    const uint64_t drain = a.drain_ns;
     // everything above only read the length arrays and the page table; inputs and the workspace
     // are touched only after the previous kernel on the stream has finished (a no-op unless
     // this grid was launched as a programmatic dependent)
@@ -287,7 +288,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tma_load_3d(&tm_q, sbase + kOffQ + hf * kHalf, q_full, hf * 64, h, (int32_t)(g.tok0 + qrow0));
         }
         int issued = 0;
-        for (int t = 0; t < n; ++t) {
+        const int n_issue = (is_v && (a.inject & kInjectStallV)) ? 0 : n;
+        for (int t = 0; t < n_issue; ++t) {
             const TileGeo tg = tile_geo(t, g.L);
             const int st = t % stages;
             // tile t goes into stage t % stages once the MMA that read tile t - stages is done
@@ -304,9 +306,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // the drain itself never raises the CTA-wide abort)
         volatile int never = 0;
         if (!is_v)
-            mbar_wait(q_full, 0, &never, tmo);
+            mbar_wait(q_full, 0, &never, drain);
         for (int t = (issued > stages ? issued - stages : 0); t < issued; ++t)
-            mbar_wait(&full[t % stages], (t / stages) & 1, &never, tmo);
+            mbar_wait(&full[t % stages], (t / stages) & 1, &never, drain);
     } else if (warp == 1 && lane == 0) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
@@ -364,7 +366,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // so tensor memory is idle before it is released)
         umma_commit(o_full);
         volatile int never = 0;
-        mbar_wait(o_full, 0, &never, tmo);
+        mbar_wait(o_full, 0, &never, drain);
     } else if (warp >= 4) {
         // ============================================================ pointwise + epilogue
         const int pt = threadIdx.x - 128;                 // 0..255

@@ -41,9 +41,15 @@ struct TcArgs {
     int32_t target_ctas;    // paged: CTAs the balanced split aims for (one per SM)
     double ln_nmax;
     float inv_n;
-    uint64_t timeout_ns;
+    uint64_t timeout_ns;    // limit of a role's wait for another role (then the CTA aborts)
+    uint64_t drain_ns;      // limit of the waits for a CTA's own copies and products in flight
     int32_t overlap_previous;   // paged: launched as a programmatic dependent of the previous kernel
+    uint32_t inject;        // test-only fault injection (kInjectStallV), 0 in normal calls
 };
+
+// inject bit: the V producer issues no load, so the first wait on a V tile runs out (tests of
+// the time-out path; every other role then aborts through its bounded waits)
+constexpr uint32_t kInjectStallV = 1u << 0;
 
 // The paged tensor-core kernel (attn_paged.cu) takes the same argument block; seq_offsets and
 // target_ctas are unused there.

@@ -384,6 +384,22 @@ int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const v
                       size_t workspace_bytes, void* stream);
 
 /*
+ * Test-only fault injection for the time-out path of the tensor-core attention kernels (bf16,
+ * D = 128, jagged and paged).  Every wait of one role of a CTA for another (a copy landing, a
+ * product completing, a buffer being released) gives up after a limit, sets HSTU_DEV_TIMEOUT
+ * in the status word and makes the CTA's other roles give up too; each role then waits for its
+ * own copies and products still in flight (with the full 2 s limit), tensor memory is released
+ * and the kernel returns.  The rows of that call are not valid; the next call is unaffected.
+ *   kind = HSTU_INJECT_STALL_V : from now on the V-tile producer issues no load, so the first
+ *          wait on a V tile runs out after wait_limit_ns (1 ms .. 2 s) instead of 2 s;
+ *   kind = 0                   : back to normal calls (wait_limit_ns ignored).
+ * Process-wide; calls already enqueued keep the setting they were launched with.  Nothing
+ * faults, traps or waits without a limit.  Not for production use.
+ */
+enum { HSTU_INJECT_STALL_V = 1 };
+int hstu_test_inject(uint32_t kind, uint64_t wait_limit_ns);
+
+/*
  * Copy `bytes` bytes from src to dst with the GPU's SMs, as one kernel on `stream`: the upload of
  * a call's inputs from pinned host memory (or the download of its outputs) done by the device
  * reading and writing host memory over the host link, instead of a DMA copy.  Either pointer
