@@ -39,6 +39,7 @@ TIER_GPU = 1
 TIER_HOST = 2
 
 FLAG_OVERLAP_PREVIOUS = 1 << 0
+FLAG_LN_PER_HEAD = 1 << 1
 
 INJECT_STALL_V = 1
 
@@ -83,6 +84,8 @@ class HstuParams(ctypes.Structure):
         ("max_pages_per_user", ctypes.c_int32),
         ("ln_eps", ctypes.c_float),
         ("flags", ctypes.c_uint32),
+        ("ln_weight", ctypes.c_void_p),
+        ("ln_bias", ctypes.c_void_p),
     ]
 
 
@@ -165,8 +168,19 @@ def _check(rc: int, what: str):
 
 
 def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, page_size: int = 0,
-           num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5, flags: int = 0) -> HstuParams:
+           num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5, flags: int = 0,
+           ln_per_head: bool = False, ln_weight=None, ln_bias=None) -> HstuParams:
+    """Mirror of hstu_attn_params.  ln_per_head / ln_weight / ln_bias select the LayerNorm-gate
+    variants (fp32 CUDA tensors of H*D elements for gamma and beta; the params object keeps them
+    alive)."""
     import torch
+
+    for name, t in (("ln_weight", ln_weight), ("ln_bias", ln_bias)):
+        if t is not None and (not t.is_cuda or t.dtype != torch.float32 or t.numel() != num_heads * head_dim
+                              or not t.is_contiguous()):
+            raise HstuError(f"{name} must be a contiguous fp32 CUDA tensor of H*D = {num_heads * head_dim} elements")
+    if ln_per_head:
+        flags |= FLAG_LN_PER_HEAD
 
     if dtype in (torch.bfloat16, "bf16"):
         dt = HSTU_DTYPE_BF16
@@ -174,8 +188,11 @@ def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, p
         dt = HSTU_DTYPE_FP32
     else:
         raise HstuError(f"unsupported dtype {dtype}")
-    return HstuParams(num_heads, head_dim, dt, num_buckets, n_max, page_size, num_pages, max_pages_per_user,
-                      ln_eps, flags)
+    p = HstuParams(num_heads, head_dim, dt, num_buckets, n_max, page_size, num_pages, max_pages_per_user,
+                   ln_eps, flags, ln_weight.data_ptr() if ln_weight is not None else None,
+                   ln_bias.data_ptr() if ln_bias is not None else None)
+    p._keep = (ln_weight, ln_bias)
+    return p
 
 
 def _ptr(t) -> Optional[int]:

@@ -100,7 +100,9 @@ static int check_params(const hstu_attn_params* p, bool paged)
         return HSTU_ERR_INVALID_ARG;
     if (!(p->ln_eps >= 0.0f) || !isfinite(p->ln_eps))
         return HSTU_ERR_INVALID_ARG;
-    if (p->flags & ~(uint32_t)HSTU_FLAG_OVERLAP_PREVIOUS)
+    if (p->flags & ~(uint32_t)(HSTU_FLAG_OVERLAP_PREVIOUS | HSTU_FLAG_LN_PER_HEAD))
+        return HSTU_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(p->ln_weight) & 3u) || (reinterpret_cast<uintptr_t>(p->ln_bias) & 3u))
         return HSTU_ERR_INVALID_ARG;
     if (p->dtype != HSTU_DTYPE_BF16 && p->dtype != HSTU_DTYPE_FP32)
         return HSTU_ERR_UNSUPPORTED;
@@ -123,6 +125,16 @@ static int check_params(const hstu_attn_params* p, bool paged)
 }
 
 static int esize_of(const hstu_attn_params* p) { return p->dtype == HSTU_DTYPE_FP32 ? 4 : 2; }
+
+static LnVariant ln_variant(const hstu_attn_params* p)
+{
+    LnVariant v;
+    v.per_head = (p->flags & HSTU_FLAG_LN_PER_HEAD) != 0;
+    v.D = p->head_dim;
+    v.gamma = p->ln_weight;
+    v.beta = p->ln_bias;
+    return v;
+}
 
 // The tensor-core kernel handles bf16, head_dim 128 and up to 1024 buckets (staged in shared memory).
 static bool use_tc(const hstu_attn_params* p)
@@ -534,7 +546,7 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
     if (rc != HSTU_OK)
         return rc;
     launch_ln_gate(part, 1, nullptr, total_tokens, params->num_heads * params->head_dim, u, out, fp32, params->ln_eps,
-                   s);
+                   ln_variant(params), s);
     return finish(s);
 }
 
@@ -554,6 +566,8 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
     int rc = check_params(params, false);
     if (rc != HSTU_OK)
         return rc;
+    if ((params->flags & HSTU_FLAG_LN_PER_HEAD) || params->ln_weight || params->ln_bias)
+        return HSTU_ERR_UNSUPPORTED;   // the backward pass implements the base LayerNorm only
     if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -706,7 +720,7 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         launch_attn_simt(a, true, fp32, B, s);
     }
     launch_ln_gate(part, splits, use_tc(params) ? counts : nullptr, total_new, params->num_heads * params->head_dim,
-                   u_new, out, fp32, params->ln_eps, s);
+                   u_new, out, fp32, params->ln_eps, ln_variant(params), s);
     return finish(s);
 }
 

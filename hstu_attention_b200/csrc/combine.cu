@@ -2,7 +2,8 @@
 //
 // Elementwise gating before the output projection (aitrends.kr summary, section
 // "HSTU의 순차 모델링"; news.bpdata.com, section "HSTU"); the library normalises the whole
-// H*D vector of a token (biased variance, eps inside the square root, no affine).
+// H*D vector of a token (biased variance, eps inside the square root, no affine), or, as
+// variants, each head's D values and/or with an affine gamma, beta before the gate.
 //
 // The attention kernels leave fp32 partial outputs o[split][token][H][D] in the workspace
 // (several splits when a user's keys were divided across CTAs; HSTU has no softmax
@@ -172,16 +173,66 @@ ln_gate_kernel_scalar(const float* __restrict__ part, int32_t S_all, const int32
     }
 }
 
+// The variants (per-head statistics and/or an affine gamma, beta before the gate): one warp per
+// token as above; the token's summed o is staged in shared memory (H*D <= 2048 floats per warp),
+// then each normalisation group -- the whole vector, or one head's D values -- gets its own
+// two-pass mean and variance.  out = ((o - mean) * rstd * gamma + beta) * u.
+template <typename T>
+__global__ void __launch_bounds__(kCombineThreads)
+ln_gate_variant_kernel(const float* __restrict__ part, int32_t S_all, const int32_t* __restrict__ counts,
+                       int64_t ntok, int32_t HD, int32_t group, const float* __restrict__ gamma,
+                       const float* __restrict__ beta, const T* __restrict__ u, T* __restrict__ out, float eps)
+{
+    extern __shared__ float xs_all[];
+    sm100::pdl_launch_dependents();
+    sm100::pdl_wait_primary();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5);
+    if (t >= ntok)
+        return;
+    float* xs = xs_all + (threadIdx.x >> 5) * HD;
+    const int32_t S = counts ? max(1, min(counts[t], S_all)) : S_all;
+    for (int e = lane; e < HD; e += 32) {
+        float acc = 0.f;
+        for (int s = 0; s < S; ++s)
+            acc += part[((int64_t)s * ntok + t) * HD + e];
+        xs[e] = acc;
+    }
+    __syncwarp();
+    for (int g0 = 0; g0 < HD; g0 += group) {
+        float sum = 0.f;
+        for (int e = g0 + lane; e < g0 + group; e += 32)
+            sum += xs[e];
+        for (int o = 16; o > 0; o >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float mean = sum / (float)group;
+        float sq = 0.f;
+        for (int e = g0 + lane; e < g0 + group; e += 32) {
+            const float d = xs[e] - mean;
+            sq += d * d;
+        }
+        for (int o = 16; o > 0; o >>= 1)
+            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+        const float rstd = 1.0f / sqrtf(sq / (float)group + eps);
+        for (int e = g0 + lane; e < g0 + group; e += 32) {
+            const int64_t idx = t * HD + e;
+            const float g = gamma ? gamma[e] : 1.0f;
+            const float b = beta ? beta[e] : 0.0f;
+            out[idx] = Elem<T>::from_float(((xs[e] - mean) * rstd * g + b) * Elem<T>::to_float(u[idx]));
+        }
+    }
+}
+
 // Launch with programmatic stream serialization: the grid may be scheduled while the
 // previous kernel on the stream is still running; the kernel waits (griddepcontrol.wait)
 // before it touches that kernel's results.
 template <typename... KArgs, typename... Args>
-static void launch_pdl(void (*kern)(KArgs...), unsigned grid, cudaStream_t stream, Args... args)
+static void launch_pdl_smem(void (*kern)(KArgs...), unsigned grid, size_t smem, cudaStream_t stream, Args... args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kCombineThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -191,14 +242,26 @@ static void launch_pdl(void (*kern)(KArgs...), unsigned grid, cudaStream_t strea
     cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+template <typename... KArgs, typename... Args>
+static void launch_pdl(void (*kern)(KArgs...), unsigned grid, cudaStream_t stream, Args... args)
+{
+    launch_pdl_smem(kern, grid, 0, stream, args...);
+}
+
 template <typename T>
 static void launch_typed(const float* part, int32_t S, const int32_t* counts, int64_t ntok, int32_t HD, const void* u,
-                         void* out, float eps, cudaStream_t stream)
+                         void* out, float eps, const LnVariant& var, cudaStream_t stream)
 {
     const int per_warp = kCombineThreads / 32;
     const unsigned grid = (unsigned)((ntok + per_warp - 1) / per_warp);
     const T* uu = static_cast<const T*>(u);
     T* oo = static_cast<T*>(out);
+    if (var.any()) {
+        const int32_t group = var.per_head ? var.D : HD;
+        launch_pdl_smem(ln_gate_variant_kernel<T>, grid, (size_t)per_warp * HD * sizeof(float), stream, part, S,
+                        counts, ntok, HD, group, var.gamma, var.beta, uu, oo, eps);
+        return;
+    }
     if (HD % 128 == 0) {
         switch (HD / 128) {
         case 1: launch_pdl(ln_gate_kernel<T, 1>, grid, stream, part, S, counts, ntok, HD, uu, oo, eps); return;
@@ -213,14 +276,14 @@ static void launch_typed(const float* part, int32_t S, const int32_t* counts, in
 }
 
 void launch_ln_gate(const float* part, int32_t S, const int32_t* counts, int64_t ntok, int32_t HD, const void* u,
-                    void* out, bool fp32, float eps, cudaStream_t stream)
+                    void* out, bool fp32, float eps, const LnVariant& var, cudaStream_t stream)
 {
     if (ntok <= 0)
         return;
     if (fp32)
-        launch_typed<float>(part, S, counts, ntok, HD, u, out, eps, stream);
+        launch_typed<float>(part, S, counts, ntok, HD, u, out, eps, var, stream);
     else
-        launch_typed<__nv_bfloat16>(part, S, counts, ntok, HD, u, out, eps, stream);
+        launch_typed<__nv_bfloat16>(part, S, counts, ntok, HD, u, out, eps, var, stream);
 }
 
 }  // namespace hstu

@@ -81,8 +81,16 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
                       int32_t P, int32_t num_pages, int32_t max_pages, int32_t max_new, void* ws,
                       cudaStream_t stream);
 // counts == nullptr: every token has S partial planes; otherwise token t has counts[t].
+// LayerNorm-gate variants (the base kernels run when none is set)
+struct LnVariant {
+    bool per_head = false;        // statistics per head (D values) instead of per token (H*D)
+    int32_t D = 0;
+    const float* gamma = nullptr; // [H*D] or null (1)
+    const float* beta = nullptr;  // [H*D] or null (0)
+    bool any() const { return per_head || gamma || beta; }
+};
 void launch_ln_gate(const float* part, int32_t S, const int32_t* counts, int64_t ntok, int32_t HD, const void* u,
-                    void* out, bool fp32, float eps, cudaStream_t stream);
+                    void* out, bool fp32, float eps, const LnVariant& var, cudaStream_t stream);
 // Backward pass of the jagged attention (attn_bwd.cu).
 struct BwdArgs {
     const void *q, *k, *v;                 // [tokens][H][D], params dtype

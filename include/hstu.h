@@ -90,6 +90,8 @@ typedef struct {
     int32_t max_pages_per_user;   /* row stride of page_table (paged calls) */
     float ln_eps;                 /* LayerNorm epsilon, e.g. 1e-5 */
     uint32_t flags;               /* HSTU_FLAG_* bits, 0 for none */
+    const float* ln_weight;       /* NULL, or a DEVICE fp32 [H*D] LayerNorm scale gamma */
+    const float* ln_bias;         /* NULL, or a DEVICE fp32 [H*D] LayerNorm shift beta */
 } hstu_attn_params;
 
 /*
@@ -106,7 +108,18 @@ typedef struct {
  * after everything before it on the stream has finished.  This is a scheduling choice of this
  * library; the pages describe no such thing.
  */
-enum { HSTU_FLAG_OVERLAP_PREVIOUS = 1u << 0 };
+enum { HSTU_FLAG_OVERLAP_PREVIOUS = 1u << 0, HSTU_FLAG_LN_PER_HEAD = 1u << 1 };
+
+/*
+ * LayerNorm-gate variants of the epilogue (forward calls; the backward pass returns
+ * HSTU_ERR_UNSUPPORTED when any is set).  The pages say only that HSTU gates elementwise before
+ * the output projection (aitrends.kr summary, section "HSTU의 순차 모델링"); these are options of
+ * this library:
+ *   HSTU_FLAG_LN_PER_HEAD : mean and variance over each head's D values of a token instead of
+ *                           its whole H*D vector;
+ *   ln_weight, ln_bias    : out = (xhat * gamma + beta) * u, gamma and beta indexed by h*D + c
+ *                           (NULL: gamma = 1, beta = 0).  4-byte aligned device arrays.
+ */
 
 /* Library version string. */
 const char* hstu_version(void);

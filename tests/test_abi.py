@@ -173,6 +173,14 @@ def test_backward_host_validation_without_gpu(lib):
     unal = list(args)
     unal[-3] = ws + 8
     assert Bw(ctypes.byref(p), *unal) == -3
+    # the LayerNorm variants exist in the forward calls only
+    assert Bw(ctypes.byref(_p(flags=hb.FLAG_LN_PER_HEAD)), *args) == -2
+    affine = _p()
+    affine.ln_weight = fake
+    assert Bw(ctypes.byref(affine), *args) == -2
+    odd = _p()
+    odd.ln_bias = fake + 2                                                # not 4-byte aligned
+    assert lib.hstu_workspace_size(ctypes.byref(odd), 1, 1, 1) == 0
 
 
 def test_binding_checks_types_before_any_call():
