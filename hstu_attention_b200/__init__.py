@@ -67,6 +67,9 @@ EXPORTED = (
     "hstu_kv_page_copy",
     "hstu_host_copy",
     "hstu_test_inject",
+    "hstu_linear_fwd",
+    "hstu_workspace_size_layer",
+    "hstu_layer_paged_fwd",
 )
 
 
@@ -151,6 +154,13 @@ def load(path: Optional[str] = None):
             lib.hstu_kv_page_copy.argtypes = [pp, vp, vp, i32, vp, vp, i32, vp, i32, vp, sz, vp]
             lib.hstu_host_copy.restype = ctypes.c_int
             lib.hstu_host_copy.argtypes = [vp, vp, sz, vp]
+            lib.hstu_linear_fwd.restype = ctypes.c_int
+            lib.hstu_linear_fwd.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, sz, vp]
+            lib.hstu_workspace_size_layer.restype = sz
+            lib.hstu_workspace_size_layer.argtypes = [pp, i32, i32, i64, i32]
+            lib.hstu_layer_paged_fwd.restype = ctypes.c_int
+            lib.hstu_layer_paged_fwd.argtypes = [pp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
+                                                 vp, sz, vp]
             lib.hstu_test_inject.restype = ctypes.c_int
             lib.hstu_test_inject.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
             _lib = lib
@@ -546,3 +556,65 @@ def test_inject(kind: int, wait_limit_ns: int = 0):
     """hstu_test_inject: test-only fault injection of the time-out path (INJECT_STALL_V: the V
     producer issues nothing and role waits give up after wait_limit_ns); kind 0 restores normal calls."""
     _check(load().hstu_test_inject(int(kind), int(wait_limit_ns)), "hstu_test_inject")
+
+
+def linear_fwd(x, w, *, activation: int = 0, workspace: Workspace, out=None, stream=None):
+    """hstu_linear_fwd: act(x w^T) for bf16 CUDA tensors x [M, K], w [N, K]; activation 1 = SiLU."""
+    import torch
+
+    for name, t in (("x", x), ("w", w)):
+        if t.dtype != torch.bfloat16 or t.dim() != 2:
+            raise HstuError(f"{name} must be a 2-D bf16 tensor")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise HstuError("x and w disagree on K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(load().hstu_linear_fwd(_ptr(x), _ptr(w), _ptr(out), M, N, K, int(activation), workspace.ptr,
+                                  workspace.nbytes, _stream(stream)), "hstu_linear_fwd")
+    return out
+
+
+class LayerWorkspace(Workspace):
+    """Device scratch of hstu_layer_paged_fwd (the paged call's workspace plus q, k, v, u and the gate)."""
+
+    def __init__(self, p: HstuParams, d_model: int, max_batch: int, max_tokens: int, max_new: int, device=None,
+                 stream=None):
+        import torch
+
+        n = load().hstu_workspace_size_layer(ctypes.byref(p), int(d_model), int(max_batch), int(max_tokens),
+                                             int(max_new))
+        if n == 0:
+            raise HstuError("hstu_workspace_size_layer: unsupported parameters")
+        self.nbytes = int(n)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        base = self.buf.data_ptr()
+        self.offset = (-base) % 256
+        self.ptr = base + self.offset
+        _check(load().hstu_workspace_init(self.ptr, self.nbytes, _stream(stream)), "hstu_workspace_init")
+
+
+def layer_paged_fwd(p: HstuParams, d_model: int, x_new, w_qkvu, w_out, k_pages, v_pages, page_table, cached_lens,
+                    new_lens, num_targets, rab, *, max_new: int, workspace: LayerWorkspace, out=None, stream=None):
+    """hstu_layer_paged_fwd: one HSTU layer (SiLU QKVU projection, append, paged attention with its
+    LayerNorm gate, output projection) for the new tokens.  Returns y [Tn, d_model] bf16."""
+    import torch
+
+    _check_args(p, elems=(("k_pages", k_pages), ("v_pages", v_pages)),
+                ints=(("page_table", page_table), ("cached_lens", cached_lens), ("new_lens", new_lens),
+                      ("num_targets", num_targets)), floats=(("rab", rab),))
+    for name, t, shape in (("x_new", x_new, (x_new.shape[0], d_model)),
+                           ("w_qkvu", w_qkvu, (4 * p.num_heads * p.head_dim, d_model)),
+                           ("w_out", w_out, (d_model, p.num_heads * p.head_dim))):
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != shape:
+            raise HstuError(f"{name} must be bf16 {shape}, got {t.dtype} {tuple(t.shape)}")
+    if out is None:
+        out = torch.empty((x_new.shape[0], d_model), dtype=torch.bfloat16, device=x_new.device)
+    B = cached_lens.shape[0]
+    rc = load().hstu_layer_paged_fwd(ctypes.byref(p), int(d_model), _ptr(x_new), _ptr(w_qkvu), _ptr(w_out),
+                                     _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(cached_lens),
+                                     _ptr(new_lens), _ptr(num_targets), _ptr(rab), _ptr(out), B, x_new.shape[0],
+                                     int(max_new), workspace.ptr, workspace.nbytes, _stream(stream))
+    _check(rc, "hstu_layer_paged_fwd")
+    return out

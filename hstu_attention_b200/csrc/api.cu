@@ -427,6 +427,122 @@ int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const v
     return finish(static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------------ projections and the layer
+
+// [rows][K] bf16 operand of the projection GEMM: box = 64 columns x 128 rows, 128B swizzle.
+static bool encode_operand(CUtensorMap* m, const void* base, int64_t rows, int32_t K)
+{
+    return encode_pages(m, base, rows, K, 128);
+}
+
+static int linear(const void* x, const void* w, __nv_bfloat16* out, int64_t M, int32_t N, int32_t K, int32_t silu,
+                  int32_t split, int64_t block_stride, void* ws, cudaStream_t s)
+{
+    CUtensorMap ta, tb;
+    if (!encode_operand(&ta, x, M, K) || !encode_operand(&tb, w, N, K))
+        return HSTU_ERR_CUDA;
+    GemmArgs g{};
+    g.M = (int32_t)M;
+    g.N = N;
+    g.K = K;
+    g.split = split;
+    g.block_stride = block_stride;
+    g.ldo = split;
+    g.out = out;
+    g.silu = silu;
+    g.ws = ws;
+    g.timeout_ns = kTimeoutNs;
+    g.drain_ns = kTimeoutNs;
+    launch_gemm_bf16(ta, tb, g, s);
+    return HSTU_OK;
+}
+
+int hstu_linear_fwd(const void* x, const void* w, void* y, int64_t M, int32_t N, int32_t K, int32_t activation,
+                    void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (M < 0 || M >= ((int64_t)1 << 31) || N <= 0 || K <= 0 || N % 128 || K % 64 || (activation != 0 && activation != 1))
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (M == 0)
+        return HSTU_OK;
+    if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y))
+        return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int rc = linear(x, w, static_cast<__nv_bfloat16*>(y), M, N, K, activation, N, 0, workspace, s);
+    return rc != HSTU_OK ? rc : finish(s);
+}
+
+static bool layer_shape_ok(const hstu_attn_params* p, int32_t d_model)
+{
+    return use_tc(p) && d_model > 0 && d_model % 128 == 0 && ((int64_t)p->num_heads * p->head_dim) % 128 == 0;
+}
+
+size_t hstu_workspace_size_layer(const hstu_attn_params* params, int32_t d_model, int32_t max_batch,
+                                 int64_t max_tokens, int32_t max_new)
+{
+    if (check_params(params, false) != HSTU_OK || !layer_shape_ok(params, d_model) || max_tokens < 0)
+        return 0;
+    const size_t attn = hstu_workspace_size(params, max_batch, max_tokens, max_new);
+    if (attn == 0)
+        return 0;
+    const size_t HD = (size_t)params->num_heads * params->head_dim;
+    const size_t act = (5 * (size_t)max_tokens * HD * 2 + 255) & ~(size_t)255;   // q, k, v, u, gated
+    return attn + act;
+}
+
+int hstu_layer_paged_fwd(const hstu_attn_params* params, int32_t d_model, const void* x_new, const void* w_qkvu,
+                         const void* w_out, void* k_pages, void* v_pages, const int32_t* page_table,
+                         const int32_t* cached_lens, const int32_t* new_lens, const int32_t* num_targets,
+                         const float* rab, void* y, int32_t B, int64_t total_new, int32_t max_new, void* workspace,
+                         size_t workspace_bytes, void* stream)
+{
+    int rc = check_params(params, true);
+    if (rc != HSTU_OK)
+        return rc;
+    if (!layer_shape_ok(params, d_model))
+        return HSTU_ERR_UNSUPPORTED;
+    if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
+        return HSTU_ERR_INVALID_ARG;
+    const size_t need = hstu_workspace_size_layer(params, d_model, B, total_new, max_new);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (B == 0 || total_new == 0)
+        return HSTU_OK;
+    if (!x_new || !w_qkvu || !w_out || !y || !aligned16(x_new) || !aligned16(w_qkvu) || !aligned16(w_out) ||
+        !aligned16(y))
+        return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t HD = (int64_t)params->num_heads * params->head_dim;
+    const size_t attn = hstu_workspace_size(params, B, total_new, max_new);
+    __nv_bfloat16* act = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(workspace) + attn);
+    __nv_bfloat16* q = act;
+    __nv_bfloat16* k = q + total_new * HD;
+    __nv_bfloat16* v = k + total_new * HD;
+    __nv_bfloat16* u = v + total_new * HD;
+    __nv_bfloat16* gated = u + total_new * HD;
+    // q, k, v, u = SiLU(x W_qkvu^T), one H*D-column block each
+    rc = linear(x_new, w_qkvu, q, total_new, (int32_t)(4 * HD), d_model, 1, (int32_t)HD, total_new * HD, workspace, s);
+    if (rc != HSTU_OK)
+        return rc;
+    // the new history tokens' K and V into the user's pages; the attention reads the new keys
+    // from k and v directly, so it does not depend on the append
+    rc = hstu_kv_append(params, k_pages, v_pages, page_table, k, v, cached_lens, new_lens, num_targets, B, total_new,
+                        max_new, workspace, attn, stream);
+    if (rc != HSTU_OK)
+        return rc;
+    hstu_attn_params pa = *params;
+    pa.flags &= ~(uint32_t)HSTU_FLAG_OVERLAP_PREVIOUS;   // inside the layer the attention starts after the append
+    rc = hstu_attn_paged_fwd(&pa, q, k, v, u, k_pages, v_pages, page_table, cached_lens, new_lens, num_targets, rab,
+                             gated, B, total_new, max_new, workspace, attn, stream);
+    if (rc != HSTU_OK)
+        return rc;
+    // y = gated W_out^T
+    rc = linear(gated, w_out, static_cast<__nv_bfloat16*>(y), total_new, d_model, (int32_t)HD, 0, d_model, 0,
+                workspace, s);
+    return rc != HSTU_OK ? rc : finish(s);
+}
+
 int hstu_test_inject(uint32_t kind, uint64_t wait_limit_ns)
 {
     if (kind & ~(uint32_t)HSTU_INJECT_STALL_V)

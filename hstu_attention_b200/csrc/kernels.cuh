@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -73,6 +74,21 @@ void launch_kv_page_copy(const void* src_k, const void* src_v, void* dst_k, void
                          cudaStream_t stream);
 
 void launch_flat_copy(void* dst, const void* src, int64_t bytes, cudaStream_t stream);
+
+// C = act(A B^T) on tensor cores (gemm.cu): A [M, K] and B [N, K] bf16 (TMA maps with 64 x 128
+// boxes), N a multiple of 128, K a multiple of 64.  Output column n goes to
+// out[(n / split) * block_stride + m * ldo + n % split].
+struct GemmArgs {
+    int32_t M, N, K;
+    int32_t split;              // columns per output block (a multiple of 128)
+    int64_t block_stride;       // elements between output blocks
+    int64_t ldo;                // elements between output rows
+    __nv_bfloat16* out;
+    int32_t silu;               // apply SiLU before rounding
+    void* ws;                   // status word (time-outs), may be null
+    uint64_t timeout_ns, drain_ns;
+};
+void launch_gemm_bf16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmArgs& g, cudaStream_t stream);
 
 void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, const void* k_new,
                       const void* v_new, const int32_t* cached_lens, const int32_t* new_lens,

@@ -275,6 +275,49 @@ int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages,
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * The HSTU layer around the attention.  The pages say that HSTU replaces softmax attention with
+ * SiLU weighting, adds a relative attention bias and gates elementwise before the output
+ * projection (aitrends.kr summary, section "HSTU의 순차 모델링"; news.bpdata.com, section
+ * "HSTU"); they do not write the projections out.  This library's reading, with no bias vectors,
+ * no residual and no input normalisation:
+ *
+ *   q, k, v, u = the four H*D-column blocks, in that order, of SiLU(x W_qkvu^T), rounded to bf16
+ *   g          = LayerNorm(attention(q, k, v)) * u      (hstu_attn_paged_fwd, bf16 out)
+ *   y          = g W_out^T
+ * ------------------------------------------------------------------------------------------ */
+
+/*
+ * y = act(x w^T) on tensor cores: x [M][K], w [N][K] (one output feature per row), y [M][N],
+ * all bf16 DEVICE arrays, 16-byte aligned; fp32 accumulation; act = 0 (none) or 1 (SiLU, applied
+ * before rounding).  N a multiple of 128, K a multiple of 64.  The workspace (>= 256 bytes,
+ * 256-byte aligned) receives HSTU_DEV_TIMEOUT if an in-kernel wait gave up.  Async on stream.
+ */
+int hstu_linear_fwd(const void* x, const void* w, void* y, int64_t M, int32_t N, int32_t K, int32_t activation,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of hstu_layer_paged_fwd: the paged call's workspace plus five bf16
+ * [max_tokens][H*D] arrays (q, k, v, u and the gated attention output).  0 if unsupported. */
+size_t hstu_workspace_size_layer(const hstu_attn_params* params, int32_t d_model, int32_t max_batch,
+                                 int64_t max_tokens, int32_t max_new);
+
+/*
+ * One HSTU layer on the paged cache hit, for the new tokens of each user:
+ *   x_new  [total_new][d_model]   the layer input of the new tokens (rows as in
+ *                                 hstu_attn_paged_fwd: user b's rows start at off_b)
+ *   w_qkvu [4*H*D][d_model], w_out [d_model][H*D]   bf16 weights, one output feature per row
+ *   y      [total_new][d_model]   the layer output
+ * The call computes q, k, v, u, appends the new history tokens' k and v to the user's pages
+ * (as hstu_kv_append; the caller advances cached_lens afterwards), runs the paged attention
+ * with its LayerNorm gate and the output projection.  Supported: bf16, D = 128, H*D and d_model
+ * multiples of 128.  The workspace holds hstu_workspace_size_layer() bytes.
+ */
+int hstu_layer_paged_fwd(const hstu_attn_params* params, int32_t d_model, const void* x_new, const void* w_qkvu,
+                         const void* w_out, void* k_pages, void* v_pages, const int32_t* page_table,
+                         const int32_t* cached_lens, const int32_t* new_lens, const int32_t* num_targets,
+                         const float* rab, void* y, int32_t B, int64_t total_new, int32_t max_new, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * KV cache management around append: a two-tier paged cache (GPU pages and pinned host pages)
  * with LRU eviction, onboard and offload, and compaction.
  *
