@@ -515,6 +515,111 @@ def bench_mixed(hb, device, steps, warmup, peaks, with_cpu):
     return line
 
 
+def bench_layer_stack(hb, device, steps, warmup, peaks, with_cpu):
+    """Sub-line: 8 whole HSTU layers on the paged cache hit, chained (layer l's output is layer
+    l+1's input): per layer the SiLU QKVU projection, the append, the paged attention with its
+    LayerNorm gate and the output projection, d_model = 512, seeded random weights per layer, each
+    layer with its own pages (the benchmark batch: 8 users, cached U[1024,4096], 16 appended +
+    64 candidates, H=4, D=128, P=32)."""
+    import torch
+
+    layers = gen.config3_paged_layers()
+    d_model = 512
+    c0 = layers[0]
+    HD = c0.H * c0.D
+    p = hb.params(c0.H, c0.D, torch.bfloat16, c0.NB, c0.n_max, page_size=c0.P, num_pages=c0.num_pages,
+                  max_pages_per_user=max(c.max_pages for c in layers))
+    shape = (c0.num_pages, c0.H, c0.P, c0.D)
+    kp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    vp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    rng = np.random.default_rng(2024)
+    meta, weights = [], []
+    for c in layers:
+        ids = torch.from_numpy(c.page_ids.astype(np.int64)).to(device)
+        kp[ids] = _to_dev(c.pool_k, device)
+        vp[ids] = _to_dev(c.pool_v, device)
+        pt = np.full((c.B, p.max_pages_per_user), -1, np.int32)
+        pt[:, :c.page_table.shape[1]] = c.page_table
+        meta.append([_to_dev(x, device) for x in (pt, c.cached_lens, c.new_lens, c.num_targets, c.rab)])
+        weights.append([_to_dev(gen._values(rng, (4 * HD, d_model), 1.0 / np.sqrt(d_model), "bf16"), device),
+                        _to_dev(gen._values(rng, (d_model, HD), 1.0 / np.sqrt(HD), "bf16"), device)])
+    Tn = int(c0.Tn)
+    max_new = max(c.max_new for c in layers)
+    x0 = _to_dev(gen._values(rng, (Tn, d_model), 1.0, "bf16"), device)
+    acts = [torch.empty((Tn, d_model), dtype=torch.bfloat16, device=device) for _ in layers]
+    ws = hb.LayerWorkspace(p, d_model, c0.B, Tn, max_new, device=device)
+
+    def step():
+        x = x0
+        for li in range(len(layers)):
+            hb.layer_paged_fwd(p, d_model, x, weights[li][0], weights[li][1], kp, vp, *meta[li][:4], meta[li][4],
+                               max_new=max_new, workspace=ws, out=acts[li])
+            x = acts[li]
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    ms = graph_ms(g, steps, torch.cuda.current_stream())
+    assert ws.status() == 0
+    # the projection GEMM alone, at the layer's shapes (tensor bound)
+    lw = hb.Workspace(p, 1, 1, 1, device=device)
+    xq = acts[0]
+    qkvu_out = torch.empty((Tn, 4 * HD), dtype=torch.bfloat16, device=device)
+    gq = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gq):
+        for _ in range(8):
+            hb.linear_fwd(xq, weights[0][0], activation=1, workspace=lw, out=qkvu_out)
+    ms_gemm = graph_ms(gq, steps, torch.cuda.current_stream()) / 8
+    proj_flops = 2 * Tn * d_model * 4 * HD + 2 * Tn * HD * d_model
+    attn_flops = sum(4 * c.D * c.H * paged_pairs(c) for c in layers)
+    flops = proj_flops * len(layers) + attn_flops
+    bf16 = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    gemm_tf = 2 * Tn * d_model * 4 * HD / (ms_gemm * 1e-3) / 1e12
+    line = {"workload": "8 chained HSTU layers on the paged cache hit (seed 1003): per layer SiLU QKVU projection "
+                        "(d_model 512 -> 4 x 512), append, paged attention + LayerNorm gate, output projection "
+                        "(512 -> 512); 8 users, cached U[1024,4096], 16 appended + 64 candidates, H=4, D=128, P=32; "
+                        "seeded random weights",
+            "new_tokens": Tn, "ms_per_step": ms, "new_tokens_per_s": Tn / (ms * 1e-3), "ms_per_layer": ms / len(layers),
+            "flops_per_step": flops, "tflops": flops / (ms * 1e-3) / 1e12,
+            "projection_gemm": {"shape": f"{Tn} x {4 * HD} x {d_model}, SiLU epilogue", "ms": ms_gemm,
+                                "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": bf16, "unit": "TFLOP/s",
+                                             "frac": gemm_tf / bf16,
+                                             "note": "5 x 16 output tiles on 148 SMs: a latency-bound small GEMM"}},
+            "launches_per_step": 6 * len(layers)}
+    if with_cpu:
+        from oracle import hstu_layer as hl
+
+        c = layers[0]
+        sub = dataclasses.replace(c, cached_lens=c.cached_lens[:1], new_lens=c.new_lens[:1],
+                                  num_targets=c.num_targets[:1], page_table=c.page_table[:1])
+        ck, cv, cpt = sub.compact_pool()
+        n0 = int(c.new_lens[0])
+        xs = gen.as_f32(gen._values(np.random.default_rng(5), (n0, d_model), 1.0, "bf16")).astype(np.float64)
+        w1 = gen.as_f32(host_bits(weights[0][0])).astype(np.float64)
+        w2 = gen.as_f32(host_bits(weights[0][1])).astype(np.float64)
+        t0 = time.perf_counter()
+        hl.layer_paged(xs, w1, w2, ck, cv, cpt, sub.cached_lens, sub.new_lens, sub.num_targets, c.rab, c.n_max)
+        dt = time.perf_counter() - t0
+        scale = len(layers) * c.B
+        line["cpu_baseline"] = {"value": Tn / (dt * scale), "unit": "new tokens/s", "kind": "oracle",
+                                "cores": __import__("oracle").default_threads(),
+                                "sample": f"one user of layer 0 ({n0} rows, {dt:.2f} s), scaled by 8 users x 8 layers"}
+    del kp, vp, ws, g, gq
+    torch.cuda.empty_cache()
+    return line
+
+
+def host_bits(t):
+    """A bf16 CUDA tensor as uint16 bit patterns on the host."""
+    import torch
+
+    return t.detach().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
 def bench_cache_ops(hb, device, steps, warmup, peaks):
     """Sub-line: the cache-management copies at the paged configuration's page shape (H=4, D=128,
     P=32, bf16: 32 KB of K and 32 KB of V per page) and the host manager's prepare latency.
@@ -689,6 +794,7 @@ def main():
     ap.add_argument("--no-long", action="store_true", help="skip the long-history sub-line")
     ap.add_argument("--no-mixed", action="store_true", help="skip the mixed-batch sub-line")
     ap.add_argument("--no-cache-ops", action="store_true", help="skip the cache-management sub-line")
+    ap.add_argument("--no-layer", action="store_true", help="skip the 8-layer HSTU stack sub-line")
     ap.add_argument("--e2e-upload", choices=("sm", "dma"), default="dma",
                     help="e2e uploads: a DMA cudaMemcpyAsync per layer (default) or hstu_host_copy (the SMs read "
                          "pinned host memory; slower here because it competes with the attention kernels)")
@@ -909,7 +1015,7 @@ def main():
             assert torch.equal(hdst.view(torch.int16), te["out"].cpu().view(torch.int16))
             assert torch.equal(te["out"].view(torch.int16), t["out"].view(torch.int16))
 
-    prefill = long_history = mixed = cache_ops = None
+    prefill = long_history = mixed = cache_ops = layer_stack = None
     if rank == 0 and not args.no_prefill:
         prefill = bench_prefill(hb, device, max(5, args.steps // 2), 3, peaks)
     with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -917,6 +1023,8 @@ def main():
         long_history = bench_long_history(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
     if rank == 0 and not args.no_mixed:
         mixed = bench_mixed(hb, device, max(3, args.steps // 4), 3, peaks, with_cpu)
+    if rank == 0 and not args.no_layer:
+        layer_stack = bench_layer_stack(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
     if rank == 0 and not args.no_cache_ops:
         cache_ops = bench_cache_ops(hb, device, max(5, args.steps // 2), 3, peaks)
 
@@ -980,6 +1088,7 @@ def main():
         "long_history": long_history,
         "mixed": mixed,
         "cache_ops": cache_ops,
+        "layer_stack": layer_stack,
     }
     print(json.dumps(line))
 
