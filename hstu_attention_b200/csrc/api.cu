@@ -666,11 +666,17 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
     return finish(s);
 }
 
+static size_t bwd_bf16_bytes(const hstu_attn_params* p, int64_t tokens)
+{
+    return ((size_t)tokens * p->num_heads * p->head_dim * 2 + 255) & ~(size_t)255;
+}
+
 size_t hstu_workspace_size_bwd(const hstu_attn_params* params, int64_t max_tokens)
 {
     if (check_params(params, false) != HSTU_OK || max_tokens < 0)
         return 0;
-    const size_t bytes = kStatusBytes + 2 * partial_bytes(params, 1, max_tokens);   // o, then d o
+    // o and its gradient (fp32), then the gradient in bf16 for the tensor-core kernels
+    const size_t bytes = kStatusBytes + 2 * partial_bytes(params, 1, max_tokens) + bwd_bf16_bytes(params, max_tokens);
     return (bytes + 255) & ~(size_t)255;
 }
 
@@ -698,7 +704,8 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
         if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(u) || !aligned16(dout) || !aligned16(dq) ||
             !aligned16(dk) || !aligned16(dv) || !aligned16(du))
             return HSTU_ERR_INVALID_ARG;
-        if (workspace_bytes < kStatusBytes + 2 * partial_bytes(params, 1, total_tokens))
+        if (workspace_bytes < kStatusBytes + 2 * partial_bytes(params, 1, total_tokens) +
+                                  bwd_bf16_bytes(params, total_tokens))
             return HSTU_ERR_WORKSPACE;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -733,7 +740,43 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
     a.max_seqlen = max_seqlen;
     a.ln_nmax = log((double)params->n_max);
     a.inv_n = (float)(1.0 / (double)params->n_max);
-    launch_jagged_bwd(a, o, u, dout, du, params->ln_eps, params->dtype == HSTU_DTYPE_FP32, s);
+    if (!use_tc(params)) {
+        launch_jagged_bwd(a, o, u, dout, du, params->ln_eps, params->dtype == HSTU_DTYPE_FP32, s);
+        return finish(s);
+    }
+    // tensor-core path: the LayerNorm-gate backward also leaves do in bf16, then dq/drab and dk/dv
+    __nv_bfloat16* dO16 = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(o) + 2 * partial_bytes(params, 1,
+                                                                                                        total_tokens));
+    BwdTcMaps m;
+    if (!encode_rows(&m.q, q, total_tokens, params->num_heads, 128) ||
+        !encode_rows(&m.k, k, total_tokens, params->num_heads, 128) ||
+        !encode_rows(&m.v, v, total_tokens, params->num_heads, 128) ||
+        !encode_rows(&m.dO, dO16, total_tokens, params->num_heads, 128))
+        return HSTU_ERR_CUDA;
+    launch_ln_gate_bwd(a, o, u, dout, du, dO16, params->ln_eps, false, s);
+    BwdTcArgs t{};
+    t.seq_offsets = seq_offsets;
+    t.num_targets = num_targets;
+    t.rab = rab;
+    t.ws = workspace;
+    t.dq = dq;
+    t.dk = dk;
+    t.dv = dv;
+    t.drab = drab;
+    t.total_tokens = total_tokens;
+    t.max_len = max_seqlen;
+    t.H = params->num_heads;
+    t.NB = params->num_buckets;
+    t.n_max = params->n_max;
+    t.B = B;
+    t.qblocks = (max_seqlen + 127) / 128;
+    t.ln_nmax = a.ln_nmax;
+    t.inv_n = a.inv_n;
+    t.timeout_ns = kTimeoutNs;
+    t.drain_ns = kTimeoutNs;
+    if (t.qblocks > 65535 || (int64_t)t.H * B >= ((int64_t)1 << 31))
+        return HSTU_ERR_UNSUPPORTED;
+    launch_bwd_tc(m, t, host_bounds(params->n_max, params->num_buckets), s);
     return finish(s);
 }
 

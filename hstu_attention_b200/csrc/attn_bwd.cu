@@ -52,7 +52,8 @@ __device__ __forceinline__ int user_of(const int32_t* off, int32_t B, int64_t t)
 template <typename T>
 __global__ void __launch_bounds__(kBwdThreads)
 ln_gate_bwd_kernel(const float* __restrict__ o, const T* __restrict__ u, const T* __restrict__ dout,
-                   float* __restrict__ du, float* __restrict__ dO, int64_t ntok, int32_t HD, float eps)
+                   float* __restrict__ du, float* __restrict__ dO, __nv_bfloat16* __restrict__ dO16, int64_t ntok,
+                   int32_t HD, float eps)
 {
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * (kBwdThreads / 32) + (threadIdx.x >> 5);
@@ -81,7 +82,10 @@ ln_gate_bwd_kernel(const float* __restrict__ o, const T* __restrict__ u, const T
     for (int e = lane; e < HD; e += 32) {
         const float xhat = (x[e] - mean) * rstd;
         const float dy = Elem<T>::to_float(dout[t * HD + e]) * Elem<T>::to_float(u[t * HD + e]);
-        dO[t * HD + e] = rstd * (dy - mdy - xhat * mdyx);
+        const float g = rstd * (dy - mdy - xhat * mdyx);
+        dO[t * HD + e] = g;
+        if (dO16)
+            dO16[t * HD + e] = __float2bfloat16_rn(g);
     }
 }
 
@@ -234,12 +238,28 @@ static void launch_typed(const BwdArgs& a, const float* o, const void* u, const 
     const int32_t HD = a.H * a.D;
     const unsigned lgrid = (unsigned)((a.total_tokens + kBwdThreads / 32 - 1) / (kBwdThreads / 32));
     ln_gate_bwd_kernel<T><<<lgrid, kBwdThreads, 0, s>>>(o, static_cast<const T*>(u), static_cast<const T*>(dout),
-                                                        du, a.dO, a.total_tokens, HD, eps);
+                                                        du, a.dO, nullptr, a.total_tokens, HD, eps);
     switch (a.D) {
     case 32: launch_pair_kernels<T, 1>(a, s); break;
     case 64: launch_pair_kernels<T, 2>(a, s); break;
     default: launch_pair_kernels<T, 4>(a, s); break;
     }
+}
+
+void launch_ln_gate_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du,
+                        __nv_bfloat16* dO16, float eps, bool fp32, cudaStream_t stream)
+{
+    if (a.total_tokens <= 0)
+        return;
+    const int32_t HD = a.H * a.D;
+    const unsigned lgrid = (unsigned)((a.total_tokens + kBwdThreads / 32 - 1) / (kBwdThreads / 32));
+    if (fp32)
+        ln_gate_bwd_kernel<float><<<lgrid, kBwdThreads, 0, stream>>>(
+            o, static_cast<const float*>(u), static_cast<const float*>(dout), du, a.dO, dO16, a.total_tokens, HD, eps);
+    else
+        ln_gate_bwd_kernel<__nv_bfloat16><<<lgrid, kBwdThreads, 0, stream>>>(
+            o, static_cast<const __nv_bfloat16*>(u), static_cast<const __nv_bfloat16*>(dout), du, a.dO, dO16,
+            a.total_tokens, HD, eps);
 }
 
 void launch_jagged_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du, float eps,

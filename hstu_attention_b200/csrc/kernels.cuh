@@ -125,6 +125,29 @@ struct BwdArgs {
 
 void launch_jagged_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du, float eps,
                        bool fp32, cudaStream_t stream);
+// Only the LayerNorm-gate backward (du, and do in fp32 and -- when dO16 is not null -- bf16).
+void launch_ln_gate_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du,
+                        __nv_bfloat16* dO16, float eps, bool fp32, cudaStream_t stream);
+
+// Backward on tensor cores (attn_bwd_tc.cu; bf16, D = 128): maps over q, k, v and the bf16
+// gradient of o, all [tokens][H][D] rows with {64, 1, 128} boxes.
+struct BwdTcMaps {
+    CUtensorMap q, k, v, dO;
+};
+struct BwdTcArgs {
+    const int32_t* seq_offsets;
+    const int32_t* num_targets;
+    const float* rab;
+    void* ws;
+    float *dq, *dk, *dv, *drab;
+    int64_t total_tokens;
+    int32_t max_len;        // max_seqlen
+    int32_t H, NB, n_max, B, qblocks;
+    double ln_nmax;
+    float inv_n;
+    uint64_t timeout_ns, drain_ns;
+};
+void launch_bwd_tc(const BwdTcMaps& m, const BwdTcArgs& a, const BucketBounds& bb, cudaStream_t stream);
 
 void launch_attn_simt(const SimtArgs& a, bool paged, bool fp32, int32_t B, cudaStream_t stream);
 // Jagged prefill on tensor cores (bf16, D = 128).
