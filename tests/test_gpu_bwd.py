@@ -101,3 +101,18 @@ def test_bwd_empty_batch_zeroes_drab(cuda_lib):
     grads = hb.jagged_bwd(p, z, z, z, z, off, None, rab, z, max_seqlen=0, workspace=ws)
     torch.cuda.synchronize()
     assert torch.all(grads[4] == 0) and ws.status() == 0
+
+
+def test_bwd_full_prefill_batch(cuda_lib):
+    """The prefill benchmark batch (8 users, lengths U[256, 4096], 64 candidates, H=4, D=128,
+    NB=128) on the tensor-core backward, every row of dq/dk/dv/du and every drab bucket against
+    the dense float64 oracle (oracle/dense_bwd.py, pinned against the pair-loop oracle)."""
+    from oracle.dense_bwd import jagged_bwd_dense
+
+    c = gen.config2_prefill()
+    dout = _dout(c, 9)
+    got, status = _run(cuda_lib, c, dout, int(c.max_seqlen))
+    assert status == 0
+    ref = jagged_bwd_dense(c.q, c.k, c.v, c.u, dout, c.seq_offsets, c.num_targets, c.rab, c.n_max, c.eps)
+    for name, g, r in zip(NAMES, got, ref):
+        _close(g, r, 1e-2, f"full prefill batch {name}")

@@ -97,3 +97,23 @@ def test_candidates_only_reach_themselves():
     g_own = oracle.hstu_jagged_bwd(c.q, c.k, c.v, c.u, only, c.seq_offsets, c.num_targets, c.rab, c.n_max)
     np.testing.assert_allclose(g_all[1][j], g_own[1][j], rtol=1e-12, atol=1e-15)   # dk
     np.testing.assert_allclose(g_all[2][j], g_own[2][j], rtol=1e-12, atol=1e-15)   # dv
+
+
+@pytest.mark.parametrize("seed,dtype", [(31, "fp32"), (32, "bf16"), (33, "bf16")])
+def test_dense_backward_equals_the_pair_loop_oracle(seed, dtype):
+    """oracle/dense_bwd.py (whole per-user matrices, library matmuls) restates the same backward as
+    the C oracle's pair loops, which finite differences pin; the two must agree to float64
+    rounding on ragged batches with candidates, including a single-token user."""
+    from oracle.dense_bwd import jagged_bwd_dense
+
+    rng = np.random.default_rng(seed)
+    lengths = [int(x) for x in rng.integers(1, 90, 3)] + [1]
+    targets = [min(int(rng.integers(0, 6)), n) for n in lengths]
+    c = gen.jagged_case(lengths, targets, H=2, D=32, NB=16, n_max=128, dtype=dtype, seed=seed, std=1.0)
+    g = rng.standard_normal(c.q.shape).astype(np.float32)
+    dout = gen.f32_to_bf16_bits(g) if dtype == "bf16" else g
+    ref = oracle.hstu_jagged_bwd(c.q, c.k, c.v, c.u, dout, c.seq_offsets, c.num_targets, c.rab, c.n_max, c.eps)
+    got = jagged_bwd_dense(c.q, c.k, c.v, c.u, dout, c.seq_offsets, c.num_targets, c.rab, c.n_max, c.eps)
+    for name, a, b in zip(("dq", "dk", "dv", "du", "drab"), got, ref):
+        scale = float(np.max(np.abs(b))) + 1e-30
+        assert np.max(np.abs(a - b)) <= 1e-10 * scale, name
