@@ -515,6 +515,65 @@ def bench_mixed(hb, device, steps, warmup, peaks, with_cpu):
     return line
 
 
+def bench_backward(hb, device, steps, warmup, peaks, with_cpu):
+    """Sub-line: the backward pass of jagged attention on the prefill batch (8 users, lengths
+    U[256,4096], 64 candidates, H=4, D=128, NB=128): o recomputed by the forward kernels, the
+    LayerNorm-gate backward, then the tensor-core dQ/drab and dK/dV kernels.  Three seeded input
+    sets rotate so consecutive calls do not find their inputs in L2."""
+    import torch
+
+    sets = []
+    for seed in (1002, 2002, 3002):
+        c = gen.config2_prefill(seed=seed)
+        dout = gen._values(np.random.default_rng(seed + 7), c.q.shape, 1.0, "bf16")
+        sets.append((c, [_to_dev(x, device) for x in (c.q, c.k, c.v, c.u, c.seq_offsets, c.num_targets, c.rab,
+                                                       dout)]))
+    c0 = sets[0][0]
+    T = max(int(c.T) for c, _ in sets)
+    ms_len = max(int(c.max_seqlen) for c, _ in sets)
+    p = hb.params(c0.H, c0.D, torch.bfloat16, c0.NB, c0.n_max, ln_eps=c0.eps)
+    ws = hb.BwdWorkspace(p, T, device=device)
+    for i in range(warmup):
+        hb.jagged_bwd(p, *sets[i % 3][1], max_seqlen=ms_len, workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        hb.jagged_bwd(p, *sets[i % 3][1], max_seqlen=ms_len, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    ms = e0.elapsed_time(e1) / steps
+    flops = float(np.mean([10 * c.D * c.H * jagged_pairs(np.diff(c.seq_offsets), c.num_targets) for c, _ in sets]))
+    tf = flops / (ms * 1e-3) / 1e12
+    bf16 = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+    line = {"workload": "backward of jagged attention on the prefill batch (seeds 1002/2002/3002 rotated): 8 users, "
+                        "lengths U[256,4096], 64 candidates, H=4, D=128, NB=128; dq, dk, dv, du (fp32) and drab",
+            "tokens": int(np.mean([c.T for c, _ in sets])), "ms_per_call": ms,
+            "algorithmic_flops_per_call": flops,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16,
+                         "note": "algorithmic FLOPs = 10 D H pairs (S recomputed, dP, dQ, dK, dV: 2.5x the forward); "
+                                 "the call also recomputes o with the forward kernels and runs the LayerNorm backward"},
+            "launches_per_call": 5}
+    if with_cpu:
+        from oracle.dense_bwd import jagged_bwd_dense
+
+        c, _ = sets[0]
+        dout = gen._values(np.random.default_rng(1009), c.q.shape, 1.0, "bf16")
+        t0 = time.perf_counter()
+        jagged_bwd_dense(c.q, c.k, c.v, c.u, dout, c.seq_offsets, c.num_targets, c.rab, c.n_max, c.eps)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": c.T / dt, "unit": "tokens/s", "kind": "oracle",
+                                "cores": os.cpu_count(),
+                                "sample": f"the whole first batch ({dt:.1f} s) on the dense float64 restatement of the "
+                                          "oracle backward (numpy matmuls on all host cores)"}
+    del ws
+    torch.cuda.empty_cache()
+    return line
+
+
 def bench_layer_stack(hb, device, steps, warmup, peaks, with_cpu):
     """Sub-line: 8 whole HSTU layers on the paged cache hit, chained (layer l's output is layer
     l+1's input): per layer the SiLU QKVU projection, the append, the paged attention with its
@@ -795,6 +854,7 @@ def main():
     ap.add_argument("--no-mixed", action="store_true", help="skip the mixed-batch sub-line")
     ap.add_argument("--no-cache-ops", action="store_true", help="skip the cache-management sub-line")
     ap.add_argument("--no-layer", action="store_true", help="skip the 8-layer HSTU stack sub-line")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward sub-line")
     ap.add_argument("--e2e-upload", choices=("sm", "dma"), default="dma",
                     help="e2e uploads: a DMA cudaMemcpyAsync per layer (default) or hstu_host_copy (the SMs read "
                          "pinned host memory; slower here because it competes with the attention kernels)")
@@ -1015,7 +1075,7 @@ def main():
             assert torch.equal(hdst.view(torch.int16), te["out"].cpu().view(torch.int16))
             assert torch.equal(te["out"].view(torch.int16), t["out"].view(torch.int16))
 
-    prefill = long_history = mixed = cache_ops = layer_stack = None
+    prefill = long_history = mixed = cache_ops = layer_stack = backward = None
     if rank == 0 and not args.no_prefill:
         prefill = bench_prefill(hb, device, max(5, args.steps // 2), 3, peaks)
     with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
@@ -1023,6 +1083,8 @@ def main():
         long_history = bench_long_history(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
     if rank == 0 and not args.no_mixed:
         mixed = bench_mixed(hb, device, max(3, args.steps // 4), 3, peaks, with_cpu)
+    if rank == 0 and not args.no_backward:
+        backward = bench_backward(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
     if rank == 0 and not args.no_layer:
         layer_stack = bench_layer_stack(hb, device, max(5, args.steps // 2), 3, peaks, with_cpu)
     if rank == 0 and not args.no_cache_ops:
@@ -1089,6 +1151,7 @@ def main():
         "mixed": mixed,
         "cache_ops": cache_ops,
         "layer_stack": layer_stack,
+        "backward": backward,
     }
     print(json.dumps(line))
 
