@@ -56,8 +56,8 @@ constexpr uint32_t kWinPad = 4;
 constexpr uint32_t kWinStride = 264;
 constexpr uint32_t kOffWin = kOffRing + 2 * kStageBytes;
 constexpr uint32_t kOffWinK = kOffWin + 4 * kWinStride * 4;  // bucket index per window position
-constexpr uint32_t kOffDiag = kOffWinK + 256 * 4;
-constexpr uint32_t kOffBsum = kOffDiag + 256 * 4;
+constexpr uint32_t kOffDiag = kOffWinK + 256 * 4;           // [8 pointwise warps][256] diagonal sums
+constexpr uint32_t kOffBsum = kOffDiag + 8 * 256 * 4;
 constexpr uint32_t kOffBounds = kOffBsum + kMaxNB * 4;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffBar = kOffRab + kMaxNB * 4;
@@ -192,8 +192,8 @@ __device__ __forceinline__ void stage_bias(const Smem& m, const BwdTcArgs& a, co
     for (int k = pt; k <= a.NB; k += 256)
         m.bounds[k] = bb.count > 0 ? bb.v[k]
                                    : (k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound_bt(k, a.ln_nmax, a.NB)));
-    if (pt < 256)
-        m.diag[pt] = 0.f;
+    for (int x = pt; x < 8 * 256; x += 256)
+        m.diag[x] = 0.f;
 }
 
 // One window position per pointwise thread: distance d(y) = dist0 + sgn * y for y = pt;
@@ -210,15 +210,20 @@ __device__ __forceinline__ void build_window(const Smem& m, int pt, int32_t dist
     m.wink[pt] = live ? k : -1;
 }
 
-// fold the tile's diagonal sums into the bucket sums and clear them (after a barrier)
+// fold the tile's diagonal sums (one private array per pointwise warp) into the bucket sums and
+// clear them (after a barrier)
 __device__ __forceinline__ void fold_diagonals(const Smem& m, int pt)
 {
     if (pt < 2 * kTile - 1) {
-        const float v = m.diag[pt];
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            v += m.diag[w * 256 + pt];
+            m.diag[w * 256 + pt] = 0.f;
+        }
         const int k = m.wink[pt];
         if (v != 0.f && k >= 0)
             atomicAdd(&m.bsum[k], v);
-        m.diag[pt] = 0.f;
     }
 }
 
@@ -351,6 +356,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int32_t lim = row_valid ? min(i + 1, g.hist) : -1;   // keys j < lim are visible, and j == i
         const int32_t diag_key = row_valid ? i : -1;
         const float inv_n = a.inv_n;
+        float* wdiag = m.diag + (warp - 4) * 256;
         bool ok = true;
         for (int t = 0; t < n; ++t) {
             const int32_t j0 = t * kTile;
@@ -383,7 +389,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const float ds = pair_terms(s, __uint_as_float(dv[e + q]), inv_n, p);
                             const bool allowed = (j < lim) | (j == diag_key);
                             ds2[q] = allowed ? ds : 0.f;
-                            atomicAdd(&m.diag[y], ds2[q]);          // no branch: masked pairs add 0
+                            // the warp's own diagonal array: in one update the 32 lanes (rows) hit 32
+                            // different diagonals; lane r + 1 hits lane r's diagonal in the next
+                            // update, so each update is fenced for the warp before the next one
+                            wdiag[y] += ds2[q];
+                            __syncwarp();
                         }
                         const __nv_bfloat162 bb2 = __floats2bfloat162_rn(ds2[0], ds2[1]);
                         packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb2);
