@@ -39,24 +39,30 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 # batch, from one `ncu --set full` capture of the attention and LayerNorm kernels (ncu flushes
 # caches, so the LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for
 # the kernel sources they were taken from (hash below); otherwise the bench reports traffic as null.
-PAGED_TRAFFIC_BYTES = 41.911808e6 + 9.728e3 + 6.407e6
-PAGED_TRAFFIC_SOURCES = "1ac49181580a31b0"
+PAGED_TRAFFIC_BYTES = 41.912576e6 + 4.352e3 + 6.407e6
+PAGED_TRAFFIC_SOURCES = "2abefd0b7776a159"
 # the same kind of capture for the jagged prefill attention kernel
-PREFILL_TRAFFIC_BYTES = 63.222528e6 + 11.850752e6
+PREFILL_TRAFFIC_BYTES = 63.22304e6 + 11.3792e6
 # long-history attention kernel: DRAM bytes of one call on the batch's first 8 users (the capture
-# size rule), 383.65 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
+# size rule), 383.73 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
 # by that ratio (traffic grows with the pages read)
-LONG_TRAFFIC_RATIO = (379.032320e6 + 4.616704e6) / 371602680
+LONG_TRAFFIC_RATIO = 383.73e6 / 371602680
+# backward dQ/drab kernel (the call's dominant kernel) on the prefill batch, per launch
+BWD_DQ_TRAFFIC_BYTES = 85.321728e6 + 14.979584e6
+BWD_TRAFFIC_SOURCES = "6f745963191d2a2d"       # hash of attn_bwd_tc.cu
+# projection GEMM (640 x 2048 x 512, SiLU) per launch
+GEMM_TRAFFIC_BYTES = 2.768384e6
+GEMM_TRAFFIC_SOURCES = "86b819eb358a215d"      # hash of gemm.cu
 
 
-def kernel_sources_hash() -> str:
-    """Hash of the two kernels' source code with comments and blank space removed (editing a
-    comment does not change the kernel the counters were taken from)."""
+def kernel_sources_hash(files=("attn_tc.cu", "attn_paged.cu", "combine.cu")) -> str:
+    """Hash of the kernels' source code with comments and blank space removed (editing a comment
+    does not change the kernel the counters were taken from)."""
     import hashlib
     import re
 
     h = hashlib.sha256()
-    for f in ("attn_tc.cu", "attn_paged.cu", "combine.cu"):
+    for f in files:
         with open(os.path.join(ROOT, "hstu_attention_b200", "csrc", f), encoding="utf-8") as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -555,7 +561,10 @@ def bench_backward(hb, device, steps, warmup, peaks, with_cpu):
             "algorithmic_flops_per_call": flops,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16,
                          "note": "algorithmic FLOPs = 10 D H pairs (S recomputed, dP, dQ, dK, dV: 2.5x the forward); "
-                                 "the call also recomputes o with the forward kernels and runs the LayerNorm backward"},
+                                 "the call also recomputes o with the forward kernels and runs the LayerNorm backward",
+                         "traffic": (BWD_DQ_TRAFFIC_BYTES if kernel_sources_hash(("attn_bwd_tc.cu",)) ==
+                                     BWD_TRAFFIC_SOURCES else None),
+                         "traffic_kernel": "bwd_dq_kernel (51 % of the call in the ncu launch list) per launch"},
             "launches_per_call": 5}
     if with_cpu:
         from oracle.dense_bwd import jagged_bwd_dense
@@ -647,6 +656,8 @@ def bench_layer_stack(hb, device, steps, warmup, peaks, with_cpu):
             "projection_gemm": {"shape": f"{Tn} x {4 * HD} x {d_model}, SiLU epilogue", "ms": ms_gemm,
                                 "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": bf16, "unit": "TFLOP/s",
                                              "frac": gemm_tf / bf16,
+                                             "traffic": (GEMM_TRAFFIC_BYTES if kernel_sources_hash(("gemm.cu",)) ==
+                                                         GEMM_TRAFFIC_SOURCES else None),
                                              "note": "5 x 16 output tiles on 148 SMs: a latency-bound small GEMM"}},
             "launches_per_step": 6 * len(layers)}
     if with_cpu:
@@ -829,6 +840,59 @@ def profile_case(case, calls):
         ws = hb.Workspace(p, c.B, c.Tn, c.max_new)
         for _ in range(calls):
             hb.paged_fwd(p, *t, kp, vp, *meta, max_new=c.max_new, workspace=ws)
+    elif case == "backward":
+        # the backward of the prefill batch (about 0.6 GB with its workspace)
+        c = gen.config2_prefill()
+        dev = torch.device("cuda", 0)
+        dout = gen._values(np.random.default_rng(9), c.q.shape, 1.0, "bf16")
+        args = [_to_dev(x, dev) for x in (c.q, c.k, c.v, c.u, c.seq_offsets, c.num_targets, c.rab, dout)]
+        p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max)
+        ws = hb.BwdWorkspace(p, c.T)
+        for _ in range(calls):
+            hb.jagged_bwd(p, *args, max_seqlen=int(c.max_seqlen), workspace=ws)
+    elif case == "layer":
+        # one HSTU layer on layer 0 of the paged batch (d_model 512): projection GEMMs + attention;
+        # the pool is compacted to the layer's pages, the appended tokens' pages included
+        c = gen.config3_paged_layers(layers=1)[0]
+        used = np.unique(c.page_table[c.page_table >= 0])
+        remap = np.full(c.num_pages, -1, dtype=np.int64)
+        remap[c.page_ids] = np.arange(c.page_ids.shape[0])
+        extra = used[remap[used] < 0]
+        remap[extra] = c.page_ids.shape[0] + np.arange(extra.shape[0])
+        pt = np.where(c.page_table >= 0, remap[np.clip(c.page_table, 0, None)], -1).astype(np.int32)
+        compact = dataclasses.replace(c, num_pages=int(c.page_ids.shape[0] + extra.shape[0]), page_table=pt,
+                                      page_ids=np.arange(c.page_ids.shape[0], dtype=np.int32))
+        dev = torch.device("cuda", 0)
+        p, _, kp, vp, L = setup_device([compact], dev)
+        t = L[0]
+        rng = np.random.default_rng(2024)
+        HD = c.H * c.D
+        w1 = _to_dev(gen._values(rng, (4 * HD, 512), 1.0 / np.sqrt(512), "bf16"), dev)
+        w2 = _to_dev(gen._values(rng, (512, HD), 1.0 / np.sqrt(HD), "bf16"), dev)
+        x = _to_dev(gen._values(rng, (int(c.Tn), 512), 1.0, "bf16"), dev)
+        ws = hb.LayerWorkspace(p, 512, c.B, int(c.Tn), c.max_new)
+        for _ in range(calls):
+            hb.layer_paged_fwd(p, 512, x, w1, w2, kp, vp, t["pt"], t["cl"], t["nl"], t["nt"], t["rab"],
+                               max_new=c.max_new, workspace=ws)
+    elif case == "cache":
+        # onboard of layer 0's cached pages from pinned host pages, and a 16,384-page in-pool move
+        c = gen.config3_paged_layers(layers=1)[0]
+        dev = torch.device("cuda", 0)
+        p = hb.params(c.H, c.D, torch.bfloat16, c.NB, c.n_max, page_size=c.P, num_pages=c.num_pages,
+                      max_pages_per_user=c.max_pages)
+        ws = hb.Workspace(p, 1, 1, 1)
+        gk = torch.zeros((c.num_pages, c.H, c.P, c.D), dtype=torch.bfloat16, device=dev)
+        gv = torch.zeros_like(gk)
+        pages = np.concatenate([c.page_table[b, :(int(c.cached_lens[b]) + c.P - 1) // c.P] for b in range(c.B)])
+        n = len(pages)
+        hk = torch.zeros((n, c.H, c.P, c.D), dtype=torch.bfloat16).pin_memory()
+        hv = torch.zeros((n, c.H, c.P, c.D), dtype=torch.bfloat16).pin_memory()
+        on = torch.from_numpy(np.stack([np.arange(n), pages], 1).astype(np.int32)).to(dev)
+        perm = np.random.default_rng(7).permutation(c.num_pages).astype(np.int32)
+        mv = torch.from_numpy(np.stack([perm[:16384], perm[16384:32768]], 1)).to(dev)
+        for _ in range(calls):
+            hb.kv_page_copy(p, hk, hv, gk, gv, on, workspace=ws)
+            hb.kv_page_copy(p, gk, gv, gk, gv, mv, workspace=ws)
     else:
         c = gen.config2_prefill()
         d = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).cuda().view(torch.bfloat16)  # noqa
@@ -859,7 +923,7 @@ def main():
                     help="e2e uploads: a DMA cudaMemcpyAsync per layer (default) or hstu_host_copy (the SMs read "
                          "pinned host memory; slower here because it competes with the attention kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["paged", "prefill", "long"], default=None,
+    ap.add_argument("--profile-case", choices=["paged", "prefill", "long", "backward", "layer", "cache"], default=None,
                     help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
     ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
