@@ -40,9 +40,11 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 # caches, so the LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for
 # the kernel sources they were taken from (hash below); otherwise the bench reports traffic as null.
 PAGED_TRAFFIC_BYTES = 41.912576e6 + 4.352e3 + 6.407e6
-PAGED_TRAFFIC_SOURCES = "2abefd0b7776a159"
+PAGED_FILES = ("attn_paged.cu", "combine.cu")
+PAGED_TRAFFIC_SOURCES = "29eef8cdbb458396"
 # the same kind of capture for the jagged prefill attention kernel
-PREFILL_TRAFFIC_BYTES = 63.22304e6 + 11.3792e6
+PREFILL_TRAFFIC_BYTES = 63.266816e6 + 13.527552e6
+PREFILL_TRAFFIC_SOURCES = "2e9b4de20c6400aa"     # hash of attn_tc.cu
 # long-history attention kernel: DRAM bytes of one call on the batch's first 8 users (the capture
 # size rule), 383.73 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
 # by that ratio (traffic grows with the pages read)
@@ -55,7 +57,7 @@ GEMM_TRAFFIC_BYTES = 2.768384e6
 GEMM_TRAFFIC_SOURCES = "86b819eb358a215d"      # hash of gemm.cu
 
 
-def kernel_sources_hash(files=("attn_tc.cu", "attn_paged.cu", "combine.cu")) -> str:
+def kernel_sources_hash(files) -> str:
     """Hash of the kernels' source code with comments and blank space removed (editing a comment
     does not change the kernel the counters were taken from)."""
     import hashlib
@@ -310,7 +312,8 @@ def bench_prefill(hb, device, steps, warmup, peaks):
     return {"workload": "jagged prefill: 8 users, lengths U[256,4096] (seed 1002), 64 candidates, H=4, D=128",
             "tokens": int(c.T), "ms_per_call": ms, "tokens_per_s": c.T / (ms * 1e-3), "tflops": tf,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
-                         "traffic": PREFILL_TRAFFIC_BYTES if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None,
+                         "traffic": (PREFILL_TRAFFIC_BYTES if kernel_sources_hash(("attn_tc.cu",)) ==
+                                     PREFILL_TRAFFIC_SOURCES else None),
                          "traffic_kernel": "attn_tc_kernel (jagged) per launch"},
             "launches_per_call": 2}
 
@@ -402,7 +405,7 @@ def bench_long_history(hb, device, steps, warmup, peaks, with_cpu):
                          "hbm_frac": gbs / hbm, "achieved_tflops": tf, "bf16_peak_tflops": bf16,
                          "tensor_frac": tf / bf16, "frac": max(gbs / hbm, tf / bf16),
                          "traffic": (LONG_TRAFFIC_RATIO * nbytes
-                                     if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None),
+                                     if kernel_sources_hash(PAGED_FILES) == PAGED_TRAFFIC_SOURCES else None),
                          "traffic_note": "ncu DRAM bytes of the attention kernel on the first 8 users, scaled to "
                                          "the full call by algorithmic bytes (1.03x algorithmic)"},
             "l2": "inputs larger than L2 (1.69 GB of distinct pages per call)"}
@@ -1196,7 +1199,7 @@ def main():
                                "concurrently on a forked stream and are not subtracted)",
                      "ms_per_call_isolated": isolated_call_ms,
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": PAGED_TRAFFIC_BYTES if kernel_sources_hash() == PAGED_TRAFFIC_SOURCES else None,
+                     "traffic": PAGED_TRAFFIC_BYTES if kernel_sources_hash(PAGED_FILES) == PAGED_TRAFFIC_SOURCES else None,
                      "peak_kind": peaks_kind, "algorithmic_bytes_per_call": mean_bytes,
                      "ms_per_call": mean_call_ms,
                      "tflops": float(np.mean(lflops)) / (mean_call_ms * 1e-3) / 1e12},

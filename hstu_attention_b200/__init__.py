@@ -89,6 +89,9 @@ class HstuParams(ctypes.Structure):
         ("flags", ctypes.c_uint32),
         ("ln_weight", ctypes.c_void_p),
         ("ln_bias", ctypes.c_void_p),
+        ("rab_time", ctypes.c_void_p),
+        ("timestamps", ctypes.c_void_p),
+        ("num_time_buckets", ctypes.c_int32),
     ]
 
 
@@ -179,7 +182,7 @@ def _check(rc: int, what: str):
 
 def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, page_size: int = 0,
            num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5, flags: int = 0,
-           ln_per_head: bool = False, ln_weight=None, ln_bias=None) -> HstuParams:
+           ln_per_head: bool = False, ln_weight=None, ln_bias=None, rab_time=None, timestamps=None) -> HstuParams:
     """Mirror of hstu_attn_params.  ln_per_head / ln_weight / ln_bias select the LayerNorm-gate
     variants (fp32 CUDA tensors of H*D elements for gamma and beta; the params object keeps them
     alive)."""
@@ -191,6 +194,14 @@ def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, p
             raise HstuError(f"{name} must be a contiguous fp32 CUDA tensor of H*D = {num_heads * head_dim} elements")
     if ln_per_head:
         flags |= FLAG_LN_PER_HEAD
+    if (rab_time is None) != (timestamps is None):
+        raise HstuError("rab_time and timestamps go together")
+    if rab_time is not None:
+        if (not rab_time.is_cuda or rab_time.dtype != torch.float32 or rab_time.dim() != 2
+                or rab_time.shape[0] != num_heads or not rab_time.is_contiguous()):
+            raise HstuError("rab_time must be a contiguous fp32 CUDA tensor [H, num_time_buckets]")
+        if not timestamps.is_cuda or timestamps.dtype != torch.int32 or not timestamps.is_contiguous():
+            raise HstuError("timestamps must be a contiguous int32 CUDA tensor, one per token")
 
     if dtype in (torch.bfloat16, "bf16"):
         dt = HSTU_DTYPE_BF16
@@ -200,8 +211,11 @@ def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, p
         raise HstuError(f"unsupported dtype {dtype}")
     p = HstuParams(num_heads, head_dim, dt, num_buckets, n_max, page_size, num_pages, max_pages_per_user,
                    ln_eps, flags, ln_weight.data_ptr() if ln_weight is not None else None,
-                   ln_bias.data_ptr() if ln_bias is not None else None)
-    p._keep = (ln_weight, ln_bias)
+                   ln_bias.data_ptr() if ln_bias is not None else None,
+                   rab_time.data_ptr() if rab_time is not None else None,
+                   timestamps.data_ptr() if timestamps is not None else None,
+                   int(rab_time.shape[1]) if rab_time is not None else 0)
+    p._keep = (ln_weight, ln_bias, rab_time, timestamps)
     return p
 
 

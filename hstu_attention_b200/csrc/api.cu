@@ -104,6 +104,10 @@ static int check_params(const hstu_attn_params* p, bool paged)
         return HSTU_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(p->ln_weight) & 3u) || (reinterpret_cast<uintptr_t>(p->ln_bias) & 3u))
         return HSTU_ERR_INVALID_ARG;
+    if (p->rab_time &&
+        (p->num_time_buckets < 1 || p->num_time_buckets > 64 || !p->timestamps ||
+         (reinterpret_cast<uintptr_t>(p->rab_time) & 3u) || (reinterpret_cast<uintptr_t>(p->timestamps) & 3u)))
+        return HSTU_ERR_INVALID_ARG;
     if (p->dtype != HSTU_DTYPE_BF16 && p->dtype != HSTU_DTYPE_FP32)
         return HSTU_ERR_UNSUPPORTED;
     if (p->head_dim != 32 && p->head_dim != 64 && p->head_dim != 128)
@@ -500,6 +504,8 @@ int hstu_layer_paged_fwd(const hstu_attn_params* params, int32_t d_model, const 
     int rc = check_params(params, true);
     if (rc != HSTU_OK)
         return rc;
+    if (params->rab_time)
+        return HSTU_ERR_UNSUPPORTED;   // the time bias exists in the jagged forward only
     if (!layer_shape_ok(params, d_model))
         return HSTU_ERR_UNSUPPORTED;
     if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
@@ -609,6 +615,9 @@ static int jagged_attention(const hstu_attn_params* params, const void* q, const
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+        a.rab_time = params->rab_time;
+        a.ts = params->timestamps;
+        a.NBT = params->num_time_buckets;
         set_waits(a);
         launch_attn_tc(m, a, host_bounds(params->n_max, params->num_buckets), B, s);
     } else {
@@ -642,6 +651,8 @@ int hstu_attn_jagged_fwd(const hstu_attn_params* params, const void* q, const vo
     int rc = check_params(params, false);
     if (rc != HSTU_OK)
         return rc;
+    if (params->rab_time && !use_tc(params))
+        return HSTU_ERR_UNSUPPORTED;   // the time bias exists on the tensor-core path only
     if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -688,8 +699,8 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
     int rc = check_params(params, false);
     if (rc != HSTU_OK)
         return rc;
-    if ((params->flags & HSTU_FLAG_LN_PER_HEAD) || params->ln_weight || params->ln_bias)
-        return HSTU_ERR_UNSUPPORTED;   // the backward pass implements the base LayerNorm only
+    if ((params->flags & HSTU_FLAG_LN_PER_HEAD) || params->ln_weight || params->ln_bias || params->rab_time)
+        return HSTU_ERR_UNSUPPORTED;   // the backward pass implements the base epilogue and bias only
     if (B < 0 || total_tokens < 0 || max_seqlen < 0 || total_tokens >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -789,6 +800,8 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
     int rc = check_params(params, true);
     if (rc != HSTU_OK)
         return rc;
+    if (params->rab_time)
+        return HSTU_ERR_UNSUPPORTED;   // the time bias exists in the jagged forward only
     if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -893,6 +906,8 @@ int hstu_attn_paged_fwd_noalloc(const hstu_attn_params* params, const void* q_ne
     int rc = check_params(params, true);
     if (rc != HSTU_OK)
         return rc;
+    if (params->rab_time)
+        return HSTU_ERR_UNSUPPORTED;   // the time bias exists in the jagged forward only
     if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (flags_out && (reinterpret_cast<uintptr_t>(flags_out) & 3u))

@@ -65,7 +65,10 @@ constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
 constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
 constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
-constexpr uint32_t kOffBar = kOffRab + kMaxNB * 4;
+constexpr int kMaxNBT = 64;                   // time buckets (second bias)
+constexpr uint32_t kOffRabT = kOffRab + kMaxNB * 4;
+constexpr uint32_t kOffTs = kOffRabT + kMaxNBT * 4;           // key timestamps of a tile, two buffers
+constexpr uint32_t kOffBar = kOffTs + 2 * kTile * 4;
 constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
@@ -116,14 +119,29 @@ __device__ __forceinline__ void bucket_search(const int32_t* bounds, int nb, int
 // bf16x2 with integer rounding (see bf16x2_round_int).
 // kMasked selects the per-column visibility test at compile time, so the full-tile loop has
 // no branch and the compiler can interleave the independent tanh chains.
-template <bool kMasked>
+// Time bucket of a timestamp difference: 0 for d <= 0, else min(nbt - 1, bit length of d).
+__device__ __forceinline__ int time_bucket(int32_t d, int nbt)
+{
+    return d <= 0 ? 0 : min(nbt - 1, 32 - __clz(d));
+}
+
+template <bool kMasked, bool kTime = false>
 __device__ __forceinline__ void silu_cols32(const uint32_t* sv, const float4* wv, uint32_t* packed, int jc,
-                                            int32_t lim, int32_t diag)
+                                            int32_t lim, int32_t diag, int32_t ts_row = 0,
+                                            const int32_t* tsk = nullptr, const float* rabt = nullptr, int nbt = 1)
 {
     const uint64_t half2 = f2pack(0.5f, 0.5f);
 #pragma unroll
     for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 bias = wv[q4];
+        float4 bias = wv[q4];
+        if (kTime) {
+            // second bias: rab_time[h][bucket(ts_i - ts_j)] / 2 (the pipeline works on halves)
+            const int4 tj = reinterpret_cast<const int4*>(tsk)[q4];
+            bias.x += rabt[time_bucket(ts_row - tj.x, nbt)];
+            bias.y += rabt[time_bucket(ts_row - tj.y, nbt)];
+            bias.z += rabt[time_bucket(ts_row - tj.z, nbt)];
+            bias.w += rabt[time_bucket(ts_row - tj.w, nbt)];
+        }
         const uint64_t xa = f2fma(f2pack(__uint_as_float(sv[4 * q4]), __uint_as_float(sv[4 * q4 + 1])), half2,
                                   f2pack(bias.x, bias.y));
         const uint64_t xb = f2fma(f2pack(__uint_as_float(sv[4 * q4 + 2]), __uint_as_float(sv[4 * q4 + 3])), half2,
@@ -167,6 +185,7 @@ __device__ int bucket_bound(int k, double ln_nmax, int nb)
     return c > 0x7ffffffe ? 0x7ffffffe : (int)c;
 }
 
+template <bool kTime>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ BucketBounds bb, const TcArgs a)
@@ -235,6 +254,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float* win = reinterpret_cast<float*>(smem + kOffWin);
     int32_t* s_bounds = reinterpret_cast<int32_t*>(smem + kOffBounds);
     float* s_rab = reinterpret_cast<float*>(smem + kOffRab);
+    float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
+    int32_t* s_ts = reinterpret_cast<int32_t*>(smem + kOffTs);
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -373,6 +394,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // rab[h]/2 and the bucket bounds (from the host, or evaluated here for many buckets)
         for (int k = pt; k < a.NB; k += 256)
             s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
+        if (kTime)
+            for (int k = pt; k < a.NBT; k += 256)
+                s_rabt[k] = 0.5f * a.rab_time[(int64_t)h * a.NBT + k];
         for (int k = pt; k <= a.NB; k += 256)
             s_bounds[k] = bb.count > 0 ? bb.v[k]
                                        : (k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB)));
@@ -387,6 +411,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool row_valid = qrow0 + r < g.N;
         const int32_t i_abs = i0 + r;
         const int32_t lim_row = row_valid ? min(i_abs + 1, g.hist) : -1;
+        const int32_t ts_row = (kTime && row_valid) ? a.ts[g.tok0 + i_abs] : 0;
         // window: this thread's 64 bias values start at index y0 = 127 - r + 64 wg; copy s holds
         // the window shifted by s floats, so (y0 - s) is a multiple of 4
         const int y0 = (kTile - 1) - r + 64 * wg;
@@ -403,6 +428,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // reader gets 16-byte aligned vectors.  Two buffers: the barrier below also orders this
             // write after every read of the buffer two tiles ago.
             float* wbuf = win + sb * (kWinBuf / 4);
+            if (kTime && pt < kTile) {
+                // the tile's key timestamps (buffer sb; ordered like the window by the barrier below)
+                const int32_t j = tg.j0 + pt;
+                s_ts[sb * kTile + pt] = j < g.L ? a.ts[g.key_row0 + j] : 0;
+            }
             {
                 int32_t d[1] = {i0 - tg.j0 + (kTile - 1) - pt};
                 int k[1];
@@ -432,17 +462,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tmem_ld_32x32b_x32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
             tmem_wait_ld();
             tmem_ld_32x32b_x32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv2[0]));
+            const int32_t* tsk = s_ts + sb * kTile + wg * 64;
             if (full)
-                silu_cols32<false>(sv, wv, packed, jc0, lim, diag);
+                silu_cols32<false, kTime>(sv, wv, packed, jc0, lim, diag, ts_row, tsk, s_rabt, a.NBT);
             else
-                silu_cols32<true>(sv, wv, packed, jc0, lim, diag);
+                silu_cols32<true, kTime>(sv, wv, packed, jc0, lim, diag, ts_row, tsk, s_rabt, a.NBT);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&s_empty[sb]);
             if (full)
-                silu_cols32<false>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag);
+                silu_cols32<false, kTime>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag, ts_row, tsk + 32, s_rabt, a.NBT);
             else
-                silu_cols32<true>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag);
+                silu_cols32<true, kTime>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag, ts_row, tsk + 32, s_rabt, a.NBT);
             // P buffer sb is free once P V of tile t - 2 completed
             if (t >= 2) {
                 ok = ok && mbar_wait_warp(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);
@@ -532,7 +563,8 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, in
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_relaxed)) {
-        cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (dev >= 0 && dev < 64)
             attr_set[dev].store(1, std::memory_order_relaxed);
     }
@@ -547,7 +579,10 @@ void launch_attn_tc(const TcMaps& m, const TcArgs& a, const BucketBounds& bb, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.overlap_previous ? 1 : 0;          // programmatic dependent launch on request
-    cudaLaunchKernelEx(&cfg, attn_tc_kernel, m.q, m.k, m.v, bb, a);
+    if (a.rab_time)
+        cudaLaunchKernelEx(&cfg, attn_tc_kernel<true>, m.q, m.k, m.v, bb, a);
+    else
+        cudaLaunchKernelEx(&cfg, attn_tc_kernel<false>, m.q, m.k, m.v, bb, a);
 }
 
 }  // namespace hstu

@@ -46,6 +46,9 @@ struct TcArgs {
     uint64_t drain_ns;      // limit of the waits for a CTA's own copies and products in flight
     int32_t overlap_previous;   // paged: launched as a programmatic dependent of the previous kernel
     uint32_t inject;        // test-only fault injection (kInjectStallV), 0 in normal calls
+    const float* rab_time;  // jagged tensor-core path: [H][NBT] second (time) bias, or null
+    const int32_t* ts;      // [tokens] timestamps (with rab_time)
+    int32_t NBT;            // time buckets
 };
 
 // inject bit: the V producer issues no load, so the first wait on a V tile runs out (tests of

@@ -92,6 +92,9 @@ typedef struct {
     uint32_t flags;               /* HSTU_FLAG_* bits, 0 for none */
     const float* ln_weight;       /* NULL, or a DEVICE fp32 [H*D] LayerNorm scale gamma */
     const float* ln_bias;         /* NULL, or a DEVICE fp32 [H*D] LayerNorm shift beta */
+    const float* rab_time;        /* NULL, or a DEVICE fp32 [H][num_time_buckets] second bias */
+    const int32_t* timestamps;    /* with rab_time: DEVICE int32 [total_tokens], one per token */
+    int32_t num_time_buckets;     /* with rab_time: 1 .. 64 */
 } hstu_attn_params;
 
 /*
@@ -109,6 +112,16 @@ typedef struct {
  * library; the pages describe no such thing.
  */
 enum { HSTU_FLAG_OVERLAP_PREVIOUS = 1u << 0, HSTU_FLAG_LN_PER_HEAD = 1u << 1 };
+
+/*
+ * Second (time) bias, jagged forward on the tensor-core path (bf16, D = 128) only; other calls
+ * return HSTU_ERR_UNSUPPORTED when rab_time is set.  HSTU's input is a timestamp-sorted stream
+ * of items and actions (aitrends.kr summary, section "HSTU의 순차 모델링"); the pages name a
+ * relative attention bias but not its form.  This library's reading of a time-based bias:
+ *     s_ij += rab_time[h][tbucket(ts_i - ts_j)],
+ *     tbucket(d) = 0 for d <= 0, else min(num_time_buckets - 1, bit length of d)
+ * (1 for d = 1, 2 for d in 2..3, 3 for 4..7, ...: log2-spaced, exact in integers).
+ */
 
 /*
  * LayerNorm-gate variants of the epilogue (forward calls; the backward pass returns

@@ -181,6 +181,15 @@ def test_backward_host_validation_without_gpu(lib):
     odd = _p()
     odd.ln_bias = fake + 2                                                # not 4-byte aligned
     assert lib.hstu_workspace_size(ctypes.byref(odd), 1, 1, 1) == 0
+    # the time bias: argument checks, and the calls that do not implement it
+    tbias = _p()
+    tbias.rab_time, tbias.timestamps, tbias.num_time_buckets = fake, fake, 16
+    assert lib.hstu_workspace_size(ctypes.byref(tbias), 1, 1, 1) > 0
+    assert Bw(ctypes.byref(tbias), *args) == -2
+    for bad in ((fake, None, 16), (fake, fake, 0), (fake, fake, 65), (fake + 2, fake, 16)):
+        tb = _p()
+        tb.rab_time, tb.timestamps, tb.num_time_buckets = bad
+        assert lib.hstu_workspace_size(ctypes.byref(tb), 1, 1, 1) == 0
 
 
 def test_binding_checks_types_before_any_call():
