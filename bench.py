@@ -599,7 +599,7 @@ def bench_layer_stack(hb, device, steps, warmup, peaks, with_cpu):
     c0 = layers[0]
     HD = c0.H * c0.D
     p = hb.params(c0.H, c0.D, torch.bfloat16, c0.NB, c0.n_max, page_size=c0.P, num_pages=c0.num_pages,
-                  max_pages_per_user=max(c.max_pages for c in layers))
+                  max_pages_per_user=max(c.max_pages for c in layers), flags=hb.FLAG_OVERLAP_PREVIOUS)
     shape = (c0.num_pages, c0.H, c0.P, c0.D)
     kp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
     vp = torch.zeros(shape, dtype=torch.bfloat16, device=device)
@@ -925,6 +925,8 @@ def main():
     ap.add_argument("--e2e-upload", choices=("sm", "dma"), default="dma",
                     help="e2e uploads: a DMA cudaMemcpyAsync per layer (default) or hstu_host_copy (the SMs read "
                          "pinned host memory; slower here because it competes with the attention kernels)")
+    ap.add_argument("--e2e-upload-streams", type=int, default=1, choices=(1, 2, 4),
+                    help="copy streams the e2e uploads alternate between (more than one measured no faster)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["paged", "prefill", "long", "backward", "layer", "cache"], default=None,
                     help="run a few calls of one workload for an ncu capture and exit (no JSON line)")
@@ -1088,7 +1090,8 @@ def main():
             with torch.cuda.graph(g):
                 run_step(hb, p, ws, kp, vp, [t], max_new, side=side)
             layer_graphs[si].append(g)
-    up = torch.cuda.Stream(device=device)
+    # uploads may alternate between copy streams (measured: no faster than one on this host link)
+    ups = [torch.cuda.Stream(device=device) for _ in range(args.e2e_upload_streams)]
     down = torch.cuda.Stream(device=device)
     ev_up = [[torch.cuda.Event() for _ in L] for _ in range(nsets)]
     ev_done = [[torch.cuda.Event() for _ in L] for _ in range(nsets)]
@@ -1101,10 +1104,12 @@ def main():
     def e2e_step(step):
         si = step % nsets
         # the step that last used this set has consumed its inputs and shipped its outputs
-        up.wait_event(ev_computed[si])
-        up.wait_event(ev_fetched[si])
-        with torch.cuda.stream(up):
-            for li in range(len(L)):
+        for up in ups:
+            up.wait_event(ev_computed[si])
+            up.wait_event(ev_fetched[si])
+        for li in range(len(L)):
+            up = ups[li % len(ups)]
+            with torch.cuda.stream(up):
                 if args.e2e_upload == "sm":
                     hb.host_copy(dev_in[si][li], host_in[li], stream=up)
                 else:
@@ -1128,7 +1133,8 @@ def main():
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    up.wait_stream(stream)                      # the first upload starts after the start event
+    for up in ups:
+        up.wait_stream(stream)                  # the first uploads start after the start event
     for s_ in range(e_steps):
         e2e_step(s_)
     stream.wait_stream(down)                    # every step's results are on the host
@@ -1207,7 +1213,7 @@ def main():
         "e2e": {"value": job_throughput(tokens, e2e_ms, world), "unit": "new tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "upload": ("hstu_host_copy (SM copy kernel reading pinned host memory)" if args.e2e_upload == "sm"
-                           else "cudaMemcpyAsync (DMA)"),
+                           else "cudaMemcpyAsync (DMA)") + f", alternating over {args.e2e_upload_streams} copy streams",
                 "mode": "one graph per layer; each layer's inputs in one pinned buffer (one upload per layer); "
                         "uploads and downloads overlap the neighbouring layers' kernels on two copy streams; "
                         "two sets of device buffers, so a step's uploads overlap the previous step"},

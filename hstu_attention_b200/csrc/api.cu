@@ -440,7 +440,7 @@ static bool encode_operand(CUtensorMap* m, const void* base, int64_t rows, int32
 }
 
 static int linear(const void* x, const void* w, __nv_bfloat16* out, int64_t M, int32_t N, int32_t K, int32_t silu,
-                  int32_t split, int64_t block_stride, void* ws, cudaStream_t s)
+                  int32_t split, int64_t block_stride, void* ws, cudaStream_t s, bool pdl = false)
 {
     CUtensorMap ta, tb;
     if (!encode_operand(&ta, x, M, K) || !encode_operand(&tb, w, N, K))
@@ -457,6 +457,7 @@ static int linear(const void* x, const void* w, __nv_bfloat16* out, int64_t M, i
     g.ws = ws;
     g.timeout_ns = kTimeoutNs;
     g.drain_ns = kTimeoutNs;
+    g.pdl = pdl ? 1 : 0;
     launch_gemm_bf16(ta, tb, g, s);
     return HSTU_OK;
 }
@@ -528,7 +529,9 @@ int hstu_layer_paged_fwd(const hstu_attn_params* params, int32_t d_model, const 
     __nv_bfloat16* u = v + total_new * HD;
     __nv_bfloat16* gated = u + total_new * HD;
     // q, k, v, u = SiLU(x W_qkvu^T), one H*D-column block each
-    rc = linear(x_new, w_qkvu, q, total_new, (int32_t)(4 * HD), d_model, 1, (int32_t)HD, total_new * HD, workspace, s);
+    const bool overlap = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) != 0;
+    rc = linear(x_new, w_qkvu, q, total_new, (int32_t)(4 * HD), d_model, 1, (int32_t)HD, total_new * HD, workspace, s,
+                overlap);
     if (rc != HSTU_OK)
         return rc;
     // the new history tokens' K and V into the user's pages; the attention reads the new keys
@@ -537,15 +540,18 @@ int hstu_layer_paged_fwd(const hstu_attn_params* params, int32_t d_model, const 
                         max_new, workspace, attn, stream);
     if (rc != HSTU_OK)
         return rc;
+    // the attention's set-up may overlap the append: before its dependency wait it reads only
+    // the length arrays, the page table and rab, which the append does not write
     hstu_attn_params pa = *params;
-    pa.flags &= ~(uint32_t)HSTU_FLAG_OVERLAP_PREVIOUS;   // inside the layer the attention starts after the append
+    pa.flags |= HSTU_FLAG_OVERLAP_PREVIOUS;
     rc = hstu_attn_paged_fwd(&pa, q, k, v, u, k_pages, v_pages, page_table, cached_lens, new_lens, num_targets, rab,
                              gated, B, total_new, max_new, workspace, attn, stream);
     if (rc != HSTU_OK)
         return rc;
     // y = gated W_out^T
+    // the output projection's set-up overlaps the LayerNorm kernel (it waits before reading gated)
     rc = linear(gated, w_out, static_cast<__nv_bfloat16*>(y), total_new, d_model, (int32_t)HD, 0, d_model, 0,
-                workspace, s);
+                workspace, s, true);
     return rc != HSTU_OK ? rc : finish(s);
 }
 

@@ -81,6 +81,10 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint64_t tmo = g.timeout_ns, drain = g.drain_ns;
+    // launched as a programmatic dependent of the previous kernel (g.pdl): the set-up above ran
+    // early; A and the outputs are touched only after that kernel has finished (a no-op otherwise)
+    pdl_launch_dependents();
+    pdl_wait_primary();
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -183,8 +187,17 @@ void launch_gemm_bf16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const Ge
         if (dev >= 0 && dev < 64)
             attr_set[dev].store(1, std::memory_order_relaxed);
     }
-    const dim3 grid((unsigned)((g.M + gm::kBM - 1) / gm::kBM), (unsigned)(g.N / gm::kBN), 1);
-    gm::gemm_bf16_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(tm_a, tm_b, g);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((g.M + gm::kBM - 1) / gm::kBM), (unsigned)(g.N / gm::kBN), 1);
+    cfg.blockDim = dim3(gm::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = gm::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = g.pdl ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, gm::gemm_bf16_kernel, tm_a, tm_b, g);
 }
 
 }  // namespace hstu

@@ -90,6 +90,7 @@ struct GemmArgs {
     int32_t silu;               // apply SiLU before rounding
     void* ws;                   // status word (time-outs), may be null
     uint64_t timeout_ns, drain_ns;
+    int32_t pdl;                // launch as a programmatic dependent of the previous kernel
 };
 void launch_gemm_bf16(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmArgs& g, cudaStream_t stream);
 
