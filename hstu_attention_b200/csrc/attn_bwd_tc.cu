@@ -61,7 +61,7 @@ constexpr uint32_t kOffBsum = kOffDiag + 8 * 256 * 4;
 constexpr uint32_t kOffBounds = kOffBsum + kMaxNB * 4;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffBar = kOffRab + kMaxNB * 4;
-constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1;     // fix, ring full/empty, sp_full, pd_full, pd_empty, acc, spare
+constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1;     // fix, ring full/empty, sp_full, pd_full, pd_empty, acc, sp_empty
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 constexpr uint32_t kTmemCols = 512;
@@ -106,7 +106,7 @@ __device__ __forceinline__ float pair_terms(float s, float dp, float inv_n, floa
 struct Smem {
     uint8_t* base;
     uint32_t sbase;
-    uint64_t *fix_full, *ring_full, *ring_empty, *sp_full, *pd_full, *pd_empty, *acc_full;
+    uint64_t *fix_full, *ring_full, *ring_empty, *sp_full, *sp_empty, *pd_full, *pd_empty, *acc_full;
     uint32_t* tmem_slot;
     volatile int* abort_flag;
     float* win;
@@ -132,6 +132,7 @@ __device__ __forceinline__ Smem carve(uint8_t* smem_raw)
     m.pd_full = bars + 6;
     m.pd_empty = bars + 7;
     m.acc_full = bars + 8;
+    m.sp_empty = bars + 9;
     m.tmem_slot = reinterpret_cast<uint32_t*>(m.base + kOffMisc);
     m.abort_flag = reinterpret_cast<volatile int*>(m.base + kOffMisc + 4);
     m.win = reinterpret_cast<float*>(m.base + kOffWin);
@@ -153,6 +154,7 @@ __device__ __forceinline__ uint32_t setup(const Smem& m, int warp)
             mbar_init(&m.ring_empty[s], 1);
         }
         mbar_init(m.sp_full, 1);
+        mbar_init(m.sp_empty, 256);
         mbar_init(m.pd_full, 256);
         mbar_init(m.pd_empty, 1);
         mbar_init(m.acc_full, 1);
@@ -296,19 +298,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_ts = idesc_bf16_f32(128, 128, 0, 1);
         bool ok = mbar_wait(m.fix_full, 0, m.abort_flag, tmo);
-        for (int t = 0; ok && t < n; ++t) {
+        // S(t) = Q K_t^T and dP(t) = dO V_t^T into their TMEM columns (stage t & 1 of the ring)
+        auto issue_sdp = [&](int t) -> bool {
             const int st = t & 1;
             const uint32_t kb = m.sbase + kOffRing + st * kStageBytes;
             const uint32_t vb = kb + kTileBytes;
-            if (!mbar_wait(&m.ring_full[st], (t >> 1) & 1, m.abort_flag, tmo)) {
-                ok = false;
-                break;
-            }
-            // the previous tile's dQ product read dS: done before S and dP are overwritten
-            if (t >= 1 && !mbar_wait(m.pd_empty, (t - 1) & 1, m.abort_flag, tmo)) {
-                ok = false;
-                break;
-            }
+            if (!mbar_wait(&m.ring_full[st], (t >> 1) & 1, m.abort_flag, tmo))
+                return false;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -323,7 +319,23 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                              smem_desc_sw128(vb + ko, 16, 1024), idesc_ss, kk > 0 ? 1u : 0u);
             }
             umma_commit(m.sp_full);
-            // dQ += dS K: A = dS (keys = K dimension, in TMEM), B = the K tile read MN-major
+            return true;
+        };
+        if (ok && n > 0)
+            ok = issue_sdp(0);
+        for (int t = 0; ok && t < n; ++t) {
+            const int st = t & 1;
+            const uint32_t kb = m.sbase + kOffRing + st * kStageBytes;
+            // the pointwise warps have S(t) and dP(t) in registers: the next tile's products may
+            // overwrite those columns while they compute dS(t)
+            if (t + 1 < n) {
+                if (!mbar_wait(m.sp_empty, t & 1, m.abort_flag, tmo) || !issue_sdp(t + 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            // dQ += dS(t) K_t: A = dS (keys = K dimension, in TMEM), B = the K tile read MN-major;
+            // it runs while the pointwise warps work on tile t + 1
             if (!mbar_wait(m.pd_full, t & 1, m.abort_flag, tmo)) {
                 ok = false;
                 break;
@@ -364,8 +376,6 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             build_window(m, pt, qrow0 - j0 + (kTile - 1), -1, nb, top);
             named_barrier_sync(4, 256);
             ok = ok && mbar_wait_warp(m.sp_full, t & 1, m.abort_flag, tmo);
-            // dS of the previous tile was read by its dQ product (pd_empty), checked by the MMA
-            // thread before it issued this tile's S: so the dS columns are free again here
             if (ok) {
                 tc_fence_after();
                 const int y0 = (kTile - 1) - r + 64 * wg;
@@ -375,6 +385,15 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_ld_32x32b_x32(tmem + lane_base + cS + 64 * wg + c0, sv);
                     tmem_ld_32x32b_x32(tmem + lane_base + cDP + 64 * wg + c0, dv);
                     tmem_wait_ld();
+                    if (c0 == 32) {
+                        // S(t) and dP(t) are in registers: the next tile's products may start
+                        tc_fence_before();
+                        mbar_arrive(m.sp_empty);
+                    } else if (t >= 1) {
+                        // dS(t - 1) must have been read by its dQ product before dS(t) is written
+                        ok = mbar_wait_warp(m.pd_empty, (t - 1) & 1, m.abort_flag, tmo);
+                        tc_fence_after();
+                    }
                     uint32_t packed[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
