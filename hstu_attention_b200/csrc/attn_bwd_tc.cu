@@ -15,8 +15,9 @@
 // bwd_dq_kernel   one CTA per (user, head, 128-query block), grid and order as the forward:
 //                 per key tile  S = Q K^T and dP = dO V^T (tcgen05, SS), pointwise dS -> bf16 in
 //                 TMEM, dQ += dS K (tcgen05, A = dS from TMEM, B = the K tile read MN-major);
-//                 drab: dS summed along the tile's 255 diagonals in shared memory, folded into
-//                 per-CTA bucket sums, one global atomic per bucket at the end.
+//                 drab: dS summed along the tile's 255 diagonals (a shuffle reduction per 32 x 32
+//                 block into per-warp arrays), folded into per-CTA bucket sums, one global atomic
+//                 per bucket at the end.
 // bwd_dkv_kernel  one CTA per (user, head, 128-key block), the blocks with most queries first:
 //                 per query tile the transposed products S^T = K Q^T and dP^T = V dO^T, pointwise
 //                 P^T and dS^T -> bf16 in TMEM (written over the S^T / dP^T columns already read),
@@ -395,9 +396,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         tc_fence_after();
                     }
                     uint32_t packed[16];
+                    float dsv[32];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        float ds2[2];
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
                             const int c = 64 * wg + c0 + e + q;
@@ -407,15 +408,27 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             float p;
                             const float ds = pair_terms(s, __uint_as_float(dv[e + q]), inv_n, p);
                             const bool allowed = (j < lim) | (j == diag_key);
-                            ds2[q] = allowed ? ds : 0.f;
-                            // the warp's own diagonal array: in one update the 32 lanes (rows) hit 32
-                            // different diagonals; lane r + 1 hits lane r's diagonal in the next
-                            // update, so each update is fenced for the warp before the next one
-                            wdiag[y] += ds2[q];
-                            __syncwarp();
+                            dsv[e + q] = allowed ? ds : 0.f;
                         }
-                        const __nv_bfloat162 bb2 = __floats2bfloat162_rn(ds2[0], ds2[1]);
+                        const __nv_bfloat162 bb2 = __floats2bfloat162_rn(dsv[e], dsv[e + 1]);
                         packed[e >> 1] = *reinterpret_cast<const uint32_t*>(&bb2);
+                    }
+                    // diagonal sums of this warp's 32 x 32 block: element (lane, k) lies on diagonal
+                    // Y0 - lane + k.  At step k lane l takes element k of lane (l + k) % 32, which lies
+                    // on diagonal Y0 - l (no wrap) or Y0 - l + 32 (wrap), so every lane ends with two
+                    // diagonal sums; the lanes' targets are all distinct, in this batch and the next
+                    {
+                        const int Y0 = (kTile - 1) - ((warp & 3) << 5) + 64 * wg + c0;
+                        float lo = 0.f, hi = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) {
+                            const float v = __shfl_sync(0xffffffffu, dsv[k], (lane + k) & 31);
+                            const bool wrap = lane + k >= 32;
+                            lo += wrap ? 0.f : v;
+                            hi += wrap ? v : 0.f;
+                        }
+                        wdiag[Y0 - lane] += lo;
+                        wdiag[Y0 - lane + 32] += hi;
                     }
                     __syncwarp();
                     tmem_st_32x32b_x16(tmem + lane_base + cDS + 32 * wg + (c0 >> 1), packed);
