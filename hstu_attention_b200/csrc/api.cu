@@ -770,7 +770,9 @@ int hstu_attn_jagged_bwd(const hstu_attn_params* params, const void* q, const vo
         !encode_rows(&m.v, v, total_tokens, params->num_heads, 128) ||
         !encode_rows(&m.dO, dO16, total_tokens, params->num_heads, 128))
         return HSTU_ERR_CUDA;
-    launch_ln_gate_bwd(a, o, u, dout, du, dO16, params->ln_eps, false, s);
+    BwdArgs a16 = a;
+    a16.dO = nullptr;                    // the tensor-core kernels read the bf16 copy only
+    launch_ln_gate_bwd(a16, o, u, dout, du, dO16, params->ln_eps, false, s);
     BwdTcArgs t{};
     t.seq_offsets = seq_offsets;
     t.num_targets = num_targets;

@@ -83,7 +83,8 @@ ln_gate_bwd_kernel(const float* __restrict__ o, const T* __restrict__ u, const T
         const float xhat = (x[e] - mean) * rstd;
         const float dy = Elem<T>::to_float(dout[t * HD + e]) * Elem<T>::to_float(u[t * HD + e]);
         const float g = rstd * (dy - mdy - xhat * mdyx);
-        dO[t * HD + e] = g;
+        if (dO)
+            dO[t * HD + e] = g;
         if (dO16)
             dO16[t * HD + e] = __float2bfloat16_rn(g);
     }

@@ -129,7 +129,7 @@ struct BwdArgs {
 
 void launch_jagged_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du, float eps,
                        bool fp32, cudaStream_t stream);
-// Only the LayerNorm-gate backward (du, and do in fp32 and -- when dO16 is not null -- bf16).
+// Only the LayerNorm-gate backward (du; do in fp32 when a.dO is not null, in bf16 when dO16 is not null).
 void launch_ln_gate_bwd(const BwdArgs& a, const float* o, const void* u, const void* dout, float* du,
                         __nv_bfloat16* dO16, float eps, bool fp32, cudaStream_t stream);
 
