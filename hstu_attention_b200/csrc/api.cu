@@ -243,27 +243,54 @@ constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;   // 8 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
-static std::atomic<void*> g_noalloc_ptr[kNoAllocMaxDevices];
 
-// Device address of g_noalloc_scratch on the current device, looked up on the first call per
-// device (the lookup may load this library's device code onto that device).
+// The array's address is looked up once per (device, CUDA context): after a device reset, or
+// under another context, the library's module is loaded again and the address changes.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CtxGetCurrentFn ctx_get_current()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
+
+struct NoAllocEntry {
+    CUcontext ctx;
+    void* ptr;
+};
+static std::mutex g_noalloc_mu;
+static NoAllocEntry g_noalloc[kNoAllocMaxDevices];
+
+// Device address of g_noalloc_scratch for the current device and context.
 static int noalloc_scratch(void** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return HSTU_ERR_CUDA;
-    if (dev >= 0 && dev < kNoAllocMaxDevices) {
-        void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-        if (p) {
-            *out = p;
-            return HSTU_OK;
-        }
+    CtxGetCurrentFn fn = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (fn)
+        fn(&ctx);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (dev >= 0 && dev < kNoAllocMaxDevices && ctx && g_noalloc[dev].ptr && g_noalloc[dev].ctx == ctx) {
+        *out = g_noalloc[dev].ptr;
+        return HSTU_OK;
     }
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
         return HSTU_ERR_CUDA;
-    if (dev >= 0 && dev < kNoAllocMaxDevices)
-        g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    if (fn)
+        fn(&ctx);                                  // the lookup may have created the context
+    if (dev >= 0 && dev < kNoAllocMaxDevices && ctx)
+        g_noalloc[dev] = NoAllocEntry{ctx, p};
     *out = p;
     return HSTU_OK;
 }

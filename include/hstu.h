@@ -254,9 +254,10 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
  * other's results: order them on one stream, or use hstu_attn_paged_fwd with separate
  * workspaces.
  *
- * The first call on each device does a one-time set-up: it looks up the array's device
- * address (cudaGetSymbolAddress on the current device), which may load the library's device
- * code onto that device.  Make that first call before any stream capture begins.
+ * The first call on each device and CUDA context does a one-time set-up: it looks up the
+ * array's device address (cudaGetSymbolAddress), which may load the library's device code onto
+ * that device; after a device reset or under another context the address is looked up again.
+ * Make the first call before any stream capture begins.
  */
 int hstu_attn_paged_fwd_noalloc(const hstu_attn_params* params, const void* q_new,
                                 const void* k_new, const void* v_new, const void* u_new,
