@@ -70,6 +70,7 @@ EXPORTED = (
     "hstu_linear_fwd",
     "hstu_workspace_size_layer",
     "hstu_layer_paged_fwd",
+    "hstu_ts_page_copy",
 )
 
 
@@ -92,6 +93,7 @@ class HstuParams(ctypes.Structure):
         ("rab_time", ctypes.c_void_p),
         ("timestamps", ctypes.c_void_p),
         ("num_time_buckets", ctypes.c_int32),
+        ("ts_pages", ctypes.c_void_p),
     ]
 
 
@@ -164,6 +166,8 @@ def load(path: Optional[str] = None):
             lib.hstu_layer_paged_fwd.restype = ctypes.c_int
             lib.hstu_layer_paged_fwd.argtypes = [pp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                  vp, sz, vp]
+            lib.hstu_ts_page_copy.restype = ctypes.c_int
+            lib.hstu_ts_page_copy.argtypes = [vp, i32, vp, i32, i32, vp, i32, vp, sz, vp]
             lib.hstu_test_inject.restype = ctypes.c_int
             lib.hstu_test_inject.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
             _lib = lib
@@ -182,7 +186,8 @@ def _check(rc: int, what: str):
 
 def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, page_size: int = 0,
            num_pages: int = 0, max_pages_per_user: int = 0, ln_eps: float = 1e-5, flags: int = 0,
-           ln_per_head: bool = False, ln_weight=None, ln_bias=None, rab_time=None, timestamps=None) -> HstuParams:
+           ln_per_head: bool = False, ln_weight=None, ln_bias=None, rab_time=None, timestamps=None,
+           ts_pages=None) -> HstuParams:
     """Mirror of hstu_attn_params.  ln_per_head / ln_weight / ln_bias select the LayerNorm-gate
     variants (fp32 CUDA tensors of H*D elements for gamma and beta; the params object keeps them
     alive)."""
@@ -194,14 +199,17 @@ def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, p
             raise HstuError(f"{name} must be a contiguous fp32 CUDA tensor of H*D = {num_heads * head_dim} elements")
     if ln_per_head:
         flags |= FLAG_LN_PER_HEAD
-    if (rab_time is None) != (timestamps is None):
-        raise HstuError("rab_time and timestamps go together")
+    if rab_time is not None and timestamps is None:
+        raise HstuError("rab_time needs timestamps")
+    if ts_pages is not None and (not ts_pages.is_cuda or ts_pages.dtype != torch.int32 or not ts_pages.is_contiguous()):
+        raise HstuError("ts_pages must be a contiguous int32 CUDA tensor [num_pages, page_size]")
+    if timestamps is not None and (not timestamps.is_cuda or timestamps.dtype != torch.int32
+                                   or not timestamps.is_contiguous()):
+        raise HstuError("timestamps must be a contiguous int32 CUDA tensor, one per token")
     if rab_time is not None:
         if (not rab_time.is_cuda or rab_time.dtype != torch.float32 or rab_time.dim() != 2
                 or rab_time.shape[0] != num_heads or not rab_time.is_contiguous()):
             raise HstuError("rab_time must be a contiguous fp32 CUDA tensor [H, num_time_buckets]")
-        if not timestamps.is_cuda or timestamps.dtype != torch.int32 or not timestamps.is_contiguous():
-            raise HstuError("timestamps must be a contiguous int32 CUDA tensor, one per token")
 
     if dtype in (torch.bfloat16, "bf16"):
         dt = HSTU_DTYPE_BF16
@@ -214,8 +222,9 @@ def params(num_heads: int, head_dim: int, dtype, num_buckets: int, n_max: int, p
                    ln_bias.data_ptr() if ln_bias is not None else None,
                    rab_time.data_ptr() if rab_time is not None else None,
                    timestamps.data_ptr() if timestamps is not None else None,
-                   int(rab_time.shape[1]) if rab_time is not None else 0)
-    p._keep = (ln_weight, ln_bias, rab_time, timestamps)
+                   int(rab_time.shape[1]) if rab_time is not None else 0,
+                   ts_pages.data_ptr() if ts_pages is not None else None)
+    p._keep = (ln_weight, ln_bias, rab_time, timestamps, ts_pages)
     return p
 
 
@@ -632,3 +641,21 @@ def layer_paged_fwd(p: HstuParams, d_model: int, x_new, w_qkvu, w_out, k_pages, 
                                      int(max_new), workspace.ptr, workspace.nbytes, _stream(stream))
     _check(rc, "hstu_layer_paged_fwd")
     return out
+
+
+def ts_page_copy(src, dst, pairs, *, workspace: Workspace, stream=None):
+    """hstu_ts_page_copy: timestamp pages [pages, P] int32 (CUDA or pinned host), page pairs[i, 0] of
+    src to page pairs[i, 1] of dst -- the timestamp side of kv_page_copy's moves."""
+    import torch
+
+    for name, t in (("src", src), ("dst", dst)):
+        if t.dtype != torch.int32 or t.dim() != 2:
+            raise HstuError(f"{name} must be int32 [pages, page_size]")
+    if src.shape[1] != dst.shape[1]:
+        raise HstuError("src and dst page sizes differ")
+    n = pairs.shape[0]
+    if n == 0:
+        return
+    _check(load().hstu_ts_page_copy(_ptr_addressable(src, "src"), src.shape[0], _ptr_addressable(dst, "dst"),
+                                    dst.shape[0], src.shape[1], _ptr_addressable(pairs, "pairs"), n, workspace.ptr,
+                                    workspace.nbytes, _stream(stream)), "hstu_ts_page_copy")

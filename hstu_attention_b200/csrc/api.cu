@@ -104,6 +104,8 @@ static int check_params(const hstu_attn_params* p, bool paged)
         return HSTU_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(p->ln_weight) & 3u) || (reinterpret_cast<uintptr_t>(p->ln_bias) & 3u))
         return HSTU_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(p->ts_pages) & 3u)
+        return HSTU_ERR_INVALID_ARG;
     if (p->rab_time &&
         (p->num_time_buckets < 1 || p->num_time_buckets > 64 || !p->timestamps ||
          (reinterpret_cast<uintptr_t>(p->rab_time) & 3u) || (reinterpret_cast<uintptr_t>(p->timestamps) & 3u)))
@@ -389,7 +391,9 @@ int hstu_kv_append(const hstu_attn_params* params, void* k_pages, void* v_pages,
         return HSTU_ERR_INVALID_ARG;
     launch_kv_append(k_pages, v_pages, page_table, k_new, v_new, cached_lens, new_lens, num_targets, B, total_new,
                      params->num_heads, params->head_dim, esize_of(params), params->page_size, params->num_pages,
-                     params->max_pages_per_user, max_new, workspace, static_cast<cudaStream_t>(stream));
+                     params->max_pages_per_user, max_new, workspace,
+                     params->ts_pages && params->timestamps ? params->ts_pages : nullptr, params->timestamps,
+                     static_cast<cudaStream_t>(stream));
     return finish(static_cast<cudaStream_t>(stream));
 }
 
@@ -591,6 +595,28 @@ int hstu_test_inject(uint32_t kind, uint64_t wait_limit_ns)
     g_inject_limit_ns.store(wait_limit_ns, std::memory_order_relaxed);
     g_inject_kind.store(kind == HSTU_INJECT_STALL_V ? kInjectStallV : 0u, std::memory_order_relaxed);
     return HSTU_OK;
+}
+
+int hstu_ts_page_copy(const int32_t* src, int32_t src_pages, int32_t* dst, int32_t dst_pages, int32_t page_size,
+                      const int32_t* pairs, int32_t n_pairs, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (n_pairs < 0 || src_pages < 0 || dst_pages < 0 || page_size < 4 || page_size % 4)
+        return HSTU_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return HSTU_ERR_WORKSPACE;
+    if (n_pairs == 0)
+        return HSTU_OK;
+    if (!src || !dst || !pairs || src_pages == 0 || dst_pages == 0 || !aligned16(src) || !aligned16(dst))
+        return HSTU_ERR_INVALID_ARG;
+    const int64_t page_bytes = (int64_t)page_size * 4;
+    const void *sp, *dp, *pr;
+    if (!device_addressable(src, (size_t)(page_bytes * src_pages), &sp) ||
+        !device_addressable(dst, (size_t)(page_bytes * dst_pages), &dp) ||
+        !device_addressable(pairs, (size_t)n_pairs * 8, &pr))
+        return HSTU_ERR_INVALID_ARG;
+    launch_kv_page_copy(sp, nullptr, const_cast<void*>(dp), nullptr, static_cast<const int32_t*>(pr), n_pairs,
+                        src_pages, dst_pages, page_bytes, workspace, static_cast<cudaStream_t>(stream));
+    return finish(static_cast<cudaStream_t>(stream));
 }
 
 int hstu_host_copy(void* dst, const void* src, size_t bytes, void* stream)
@@ -835,8 +861,8 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
     int rc = check_params(params, true);
     if (rc != HSTU_OK)
         return rc;
-    if (params->rab_time)
-        return HSTU_ERR_UNSUPPORTED;   // the time bias exists in the jagged forward only
+    if (params->rab_time && (!use_tc(params) || !params->ts_pages))
+        return HSTU_ERR_UNSUPPORTED;   // the time bias: tensor-core path, cached timestamps in ts_pages
     if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -898,6 +924,10 @@ int hstu_attn_paged_fwd(const hstu_attn_params* params, const void* q_new, const
         a.ln_nmax = ln_nmax;
         a.inv_n = (float)(1.0 / (double)params->n_max);
         a.overlap_previous = (params->flags & HSTU_FLAG_OVERLAP_PREVIOUS) ? 1 : 0;
+        a.rab_time = params->rab_time;
+        a.ts = params->timestamps;
+        a.ts_pages = params->ts_pages;
+        a.NBT = params->num_time_buckets;
         set_waits(a);
         launch_attn_paged(m, a, host_bounds(params->n_max, params->num_buckets), num_sms(), s);
     } else {
@@ -941,8 +971,8 @@ int hstu_attn_paged_fwd_noalloc(const hstu_attn_params* params, const void* q_ne
     int rc = check_params(params, true);
     if (rc != HSTU_OK)
         return rc;
-    if (params->rab_time)
-        return HSTU_ERR_UNSUPPORTED;   // the time bias exists in the jagged forward only
+    if (params->rab_time && (!use_tc(params) || !params->ts_pages))
+        return HSTU_ERR_UNSUPPORTED;   // the time bias: tensor-core path, cached timestamps in ts_pages
     if (B < 0 || total_new < 0 || max_new < 0 || total_new >= ((int64_t)1 << 31))
         return HSTU_ERR_INVALID_ARG;
     if (flags_out && (reinterpret_cast<uintptr_t>(flags_out) & 3u))

@@ -76,7 +76,10 @@ constexpr uint32_t kRingBytes = (kKStages + kVStages) * kTileBytes;
 constexpr uint32_t kOffBounds = kOffWin + 4 * kWinBuf;    // two windows per warpgroup
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffPages = kOffRab + kMaxNB * 4;
-constexpr uint32_t kOffBar = kOffPages + kMaxPageIds * 4;
+constexpr int kMaxNBT = 64;                   // time buckets (second bias)
+constexpr uint32_t kOffRabT = kOffPages + kMaxPageIds * 4;
+constexpr uint32_t kOffTs = kOffRabT + kMaxNBT * 4;           // key timestamps: a buffer per window
+constexpr uint32_t kOffBar = kOffTs + 4 * kKeys * 4;
 constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
@@ -325,14 +328,29 @@ __device__ int bucket_bound_dev(int k, double ln_nmax, int nb)
 // SiLU weights of 32 consecutive key columns of one query row: x/2 = S/2 + bias (bias holds
 // rab/2), w = x/2 (1 + tanh(x/2)), masked to 0 where the key is not visible (j < lim or
 // j == diag), packed to bf16 pairs with integer rounding (see bf16x2_round_int).
-template <bool kMasked>
+// Time bucket of a timestamp difference: 0 for d <= 0, else min(nbt - 1, bit length of d).
+__device__ __forceinline__ int time_bucket(int32_t d, int nbt)
+{
+    return d <= 0 ? 0 : min(nbt - 1, 32 - __clz(d));
+}
+
+template <bool kMasked, bool kTime = false>
 __device__ __forceinline__ void silu_cols32(const uint32_t* sv, const float4* wv, uint32_t* packed, int jc,
-                                            int32_t lim, int32_t diag)
+                                            int32_t lim, int32_t diag, int32_t ts_row = 0,
+                                            const int32_t* tsk = nullptr, const float* rabt = nullptr, int nbt = 1)
 {
     const uint64_t half2 = f2pack(0.5f, 0.5f);
 #pragma unroll
     for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 bias = wv[q4];
+        float4 bias = wv[q4];
+        if (kTime) {
+            // second bias: rab_time[h][bucket(ts_i - ts_j)] / 2 (the pipeline works on halves)
+            const int4 tj = reinterpret_cast<const int4*>(tsk)[q4];
+            bias.x += rabt[time_bucket(ts_row - tj.x, nbt)];
+            bias.y += rabt[time_bucket(ts_row - tj.y, nbt)];
+            bias.z += rabt[time_bucket(ts_row - tj.z, nbt)];
+            bias.w += rabt[time_bucket(ts_row - tj.w, nbt)];
+        }
         const uint64_t xa = f2fma(f2pack(__uint_as_float(sv[4 * q4]), __uint_as_float(sv[4 * q4 + 1])), half2,
                                   f2pack(bias.x, bias.y));
         const uint64_t xb = f2fma(f2pack(__uint_as_float(sv[4 * q4 + 2]), __uint_as_float(sv[4 * q4 + 3])), half2,
@@ -381,6 +399,7 @@ __device__ __forceinline__ void prefetch_tile(const CUtensorMap* tm_pages, const
     }
 }
 
+template <bool kTime>
 __global__ void __maxnreg__(128)
 attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
@@ -411,6 +430,8 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     int32_t* s_bounds = reinterpret_cast<int32_t*>(smem + kOffBounds);
     float* s_rab = reinterpret_cast<float*>(smem + kOffRab);
     int32_t* s_pages = reinterpret_cast<int32_t*>(smem + kOffPages);
+    float* s_rabt = reinterpret_cast<float*>(smem + kOffRabT);
+    int32_t* s_ts = reinterpret_cast<int32_t*>(smem + kOffTs);
 
     // ---------------------------------------------------------------- plan and set-up
     // only the length arrays and the page table are read before the dependency wait
@@ -663,6 +684,9 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int pt_id = threadIdx.x - 128;
         for (int k = pt_id; k < a.NB; k += 256)
             s_rab[k] = 0.5f * a.rab[(int64_t)p.h * a.NB + k];
+        if (kTime)
+            for (int k = pt_id; k < a.NBT; k += 256)
+                s_rabt[k] = 0.5f * a.rab_time[(int64_t)p.h * a.NBT + k];
         for (int k = pt_id; k <= a.NB; k += 256)
             s_bounds[k] = bb.count > 0 ? bb.v[k]
                                        : (k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound_dev(k, a.ln_nmax, a.NB)));
@@ -680,6 +704,7 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const bool row_valid = r < nq;
         const int32_t i_abs = i0 + r;
         const int32_t lim_row = row_valid ? min(i_abs + 1, p.hist) : -1;
+        const int32_t ts_row = (kTime && row_valid) ? a.ts[p.off + qrow0 + r] : 0;   // a new token's timestamp
         const int y0 = (kKeys - 1) - r;                   // window index of (row r, key column 0)
         const int wsel = y0 & 3;
         const int woff = wsel * kWinStride + kWinPad + (y0 - wsel);
@@ -693,6 +718,25 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // 4-float pad, so every reader gets 16-byte aligned vectors.  Two buffers per warpgroup:
             // the barrier below also orders this write after every read of the buffer two tiles ago.
             float* wbuf = win + (2 * wg + ((t >> 1) & 1)) * (kWinBuf / 4);
+            int32_t* tsbuf = s_ts + (2 * wg + ((t >> 1) & 1)) * kKeys;
+            if (kTime) {
+                // the tile's key timestamps: cached keys from the timestamp pages (same page ids as
+                // K and V), new keys from the new tokens' timestamps; past the valid keys 0
+                const int32_t j = tg.j0 + wt;
+                int32_t tsv = 0;
+                if (wt < tg.nvalid) {
+                    if (tg.cached) {
+                        const int32_t lp = j / P;
+                        const int32_t rel = lp - lp_begin;
+                        int32_t pg = rel < kMaxPageIds ? s_pages[rel] : a.page_table[(int64_t)p.b * a.max_pages + lp];
+                        if (pg >= 0 && pg < a.num_pages)
+                            tsv = a.ts_pages[(int64_t)pg * P + (j - lp * P)];
+                    } else {
+                        tsv = a.ts[p.off + (j - p.C)];
+                    }
+                }
+                tsbuf[wt] = tsv;
+            }
             {
                 const int32_t dist0 = i0 - tg.j0 + (kKeys - 1);
                 int32_t d[2];
@@ -741,9 +785,11 @@ attn_paged_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     uint32_t packed[16];
                     if (full)
-                        silu_cols32<false>(sv, wv + (c0 >> 2), packed, tg.j0 + c0, lim, diag);
+                        silu_cols32<false, kTime>(sv, wv + (c0 >> 2), packed, tg.j0 + c0, lim, diag, ts_row,
+                                                  tsbuf + c0, s_rabt, a.NBT);
                     else
-                        silu_cols32<true>(sv, wv + (c0 >> 2), packed, tg.j0 + c0, lim, diag);
+                        silu_cols32<true, kTime>(sv, wv + (c0 >> 2), packed, tg.j0 + c0, lim, diag, ts_row,
+                                                 tsbuf + c0, s_rabt, a.NBT);
                     tmem_st_32x32b_x16(pcol + (c0 >> 1), packed);
                 }
             } else {
@@ -831,7 +877,9 @@ void launch_attn_paged(const TcMaps& m, const PagedArgs& a, const BucketBounds& 
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_relaxed)) {
-        cudaFuncSetAttribute(pg::attn_paged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pg::kSmemBytes);
+        cudaFuncSetAttribute(pg::attn_paged_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pg::kSmemBytes);
+        cudaFuncSetAttribute(pg::attn_paged_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, pg::kSmemBytes);
         if (dev >= 0 && dev < 64)
             attr_set[dev].store(1, std::memory_order_relaxed);
     }
@@ -855,7 +903,10 @@ void launch_attn_paged(const TcMaps& m, const PagedArgs& a, const BucketBounds& 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.overlap_previous ? 1 : 0;
-    cudaLaunchKernelEx(&cfg, pg::attn_paged_kernel, m.q, m.k, m.v, m.kp, m.vp, bb, a);
+    if (a.rab_time)
+        cudaLaunchKernelEx(&cfg, pg::attn_paged_kernel<true>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
+    else
+        cudaLaunchKernelEx(&cfg, pg::attn_paged_kernel<false>, m.q, m.k, m.v, m.kp, m.vp, bb, a);
 }
 
 }  // namespace hstu

@@ -47,7 +47,8 @@ struct TcArgs {
     int32_t overlap_previous;   // paged: launched as a programmatic dependent of the previous kernel
     uint32_t inject;        // test-only fault injection (kInjectStallV), 0 in normal calls
     const float* rab_time;  // jagged tensor-core path: [H][NBT] second (time) bias, or null
-    const int32_t* ts;      // [tokens] timestamps (with rab_time)
+    const int32_t* ts;      // [tokens] timestamps (with rab_time): all tokens (jagged) or new tokens (paged)
+    const int32_t* ts_pages;    // paged: [num_pages][P] timestamps of the cached tokens
     int32_t NBT;            // time buckets
 };
 
@@ -99,7 +100,7 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
                       const int32_t* num_targets, int32_t B, int64_t total_new, int32_t H, int32_t D,
                       int32_t esize,
                       int32_t P, int32_t num_pages, int32_t max_pages, int32_t max_new, void* ws,
-                      cudaStream_t stream);
+                      int32_t* ts_pages, const int32_t* ts_new, cudaStream_t stream);
 // counts == nullptr: every token has S partial planes; otherwise token t has counts[t].
 // LayerNorm-gate variants (the base kernels run when none is set)
 struct LnVariant {

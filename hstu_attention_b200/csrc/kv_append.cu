@@ -23,7 +23,7 @@ kv_append_kernel(uint4* __restrict__ k_pages, uint4* __restrict__ v_pages, const
                  const int32_t* __restrict__ cached_lens, const int32_t* __restrict__ new_lens,
                  const int32_t* __restrict__ num_targets, int64_t total_new, int32_t H,
                  int32_t row_chunks /* D*esize/16 */, int32_t P, int32_t num_pages, int32_t max_pages,
-                 int32_t max_new, void* ws)
+                 int32_t max_new, void* ws, int32_t* __restrict__ ts_pages, const int32_t* __restrict__ ts_new)
 {
     __shared__ int64_t s_off;
     __shared__ int32_t s_ok;
@@ -61,6 +61,11 @@ kv_append_kernel(uint4* __restrict__ k_pages, uint4* __restrict__ v_pages, const
             }
         }
         s_pages[threadIdx.x] = page;
+        if (ts_pages && page >= 0) {
+            // the token's timestamp goes beside its K and V (slot for slot)
+            const int64_t pos = (int64_t)C + t;
+            ts_pages[(int64_t)page * P + pos % P] = ts_new[s_off + t];
+        }
     }
     __syncthreads();
     const int64_t off = s_off;
@@ -88,7 +93,7 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
                       const int32_t* num_targets, int32_t B, int64_t total_new, int32_t H, int32_t D,
                       int32_t esize,
                       int32_t P, int32_t num_pages, int32_t max_pages, int32_t max_new, void* ws,
-                      cudaStream_t stream)
+                      int32_t* ts_pages, const int32_t* ts_new, cudaStream_t stream)
 {
     if (B <= 0 || max_new <= 0)
         return;
@@ -96,7 +101,7 @@ void launch_kv_append(void* k_pages, void* v_pages, const int32_t* page_table, c
     kv_append_kernel<<<grid, kAppendThreads, 0, stream>>>(
         static_cast<uint4*>(k_pages), static_cast<uint4*>(v_pages), page_table, static_cast<const uint4*>(k_new),
         static_cast<const uint4*>(v_new), cached_lens, new_lens, num_targets, total_new, H, D * esize / 16, P,
-        num_pages, max_pages, max_new, ws);
+        num_pages, max_pages, max_new, ws, ts_pages, ts_new);
 }
 
 }  // namespace hstu

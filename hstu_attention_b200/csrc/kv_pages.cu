@@ -59,7 +59,9 @@ void launch_kv_page_copy(const void* src_k, const void* src_v, void* dst_k, void
         return;
     const int64_t page_vecs = page_bytes / 16;
     const int64_t per_block = (int64_t)kCopyThreads * kCopyUnroll;
-    dim3 grid((unsigned)((page_vecs + per_block - 1) / per_block), (unsigned)(n_pairs < 65535 ? n_pairs : 65535), 2);
+    // z = the pools copied: K and V, or one pool when src_v is null (the timestamp pages)
+    dim3 grid((unsigned)((page_vecs + per_block - 1) / per_block), (unsigned)(n_pairs < 65535 ? n_pairs : 65535),
+              src_v ? 2 : 1);
     kv_page_copy_kernel<<<grid, kCopyThreads, 0, stream>>>(
         static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v), static_cast<uint4*>(dst_k),
         static_cast<uint4*>(dst_v), pairs, n_pairs, src_pages, dst_pages, page_vecs, ws);

@@ -93,8 +93,11 @@ typedef struct {
     const float* ln_weight;       /* NULL, or a DEVICE fp32 [H*D] LayerNorm scale gamma */
     const float* ln_bias;         /* NULL, or a DEVICE fp32 [H*D] LayerNorm shift beta */
     const float* rab_time;        /* NULL, or a DEVICE fp32 [H][num_time_buckets] second bias */
-    const int32_t* timestamps;    /* with rab_time: DEVICE int32 [total_tokens], one per token */
+    const int32_t* timestamps;    /* DEVICE int32, one per token: all tokens (jagged) or the new
+                                     tokens (paged, kv_append); used with rab_time / ts_pages */
     int32_t num_time_buckets;     /* with rab_time: 1 .. 64 */
+    int32_t* ts_pages;            /* paged calls: NULL, or DEVICE int32 [num_pages][P] timestamps of
+                                     the cached tokens, slot for slot beside the K/V pages */
 } hstu_attn_params;
 
 /*
@@ -114,8 +117,11 @@ typedef struct {
 enum { HSTU_FLAG_OVERLAP_PREVIOUS = 1u << 0, HSTU_FLAG_LN_PER_HEAD = 1u << 1 };
 
 /*
- * Second (time) bias, jagged forward on the tensor-core path (bf16, D = 128) only; other calls
- * return HSTU_ERR_UNSUPPORTED when rab_time is set.  HSTU's input is a timestamp-sorted stream
+ * Second (time) bias, on the tensor-core path (bf16, D = 128) of the jagged and paged forward
+ * calls (hstu_attn_paged_fwd and _noalloc read the cached tokens' timestamps from ts_pages);
+ * the backward, the layer call and the CUDA-core paths return HSTU_ERR_UNSUPPORTED when rab_time
+ * is set.  hstu_kv_append writes the appended tokens' timestamps into ts_pages when ts_pages and
+ * timestamps are set.  HSTU's input is a timestamp-sorted stream
  * of items and actions (aitrends.kr summary, section "HSTU의 순차 모델링"); the pages name a
  * relative attention bias but not its form.  This library's reading of a time-based bias:
  *     s_ij += rab_time[h][tbucket(ts_i - ts_j)],
@@ -468,6 +474,15 @@ int hstu_kv_page_copy(const hstu_attn_params* params, const void* src_k, const v
  */
 enum { HSTU_INJECT_STALL_V = 1 };
 int hstu_test_inject(uint32_t kind, uint64_t wait_limit_ns);
+
+/*
+ * Copy whole timestamp pages ([pages][page_size] int32) for i < n_pairs: page pairs[2i] of src to
+ * page pairs[2i+1] of dst -- the timestamp side of an onboard, offload or compaction move made by
+ * hstu_kv_page_copy.  Pools may be device memory or pinned host memory, as there; page_size a
+ * multiple of 4; bad page ids are skipped and set HSTU_DEV_BAD_PAGE in the workspace.
+ */
+int hstu_ts_page_copy(const int32_t* src, int32_t src_pages, int32_t* dst, int32_t dst_pages, int32_t page_size,
+                      const int32_t* pairs, int32_t n_pairs, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Copy `bytes` bytes from src to dst with the GPU's SMs, as one kernel on `stream`: the upload of
