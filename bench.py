@@ -39,22 +39,22 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 # batch, from one `ncu --set full` capture of the attention and LayerNorm kernels (ncu flushes
 # caches, so the LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for
 # the kernel sources they were taken from (hash below); otherwise the bench reports traffic as null.
-PAGED_TRAFFIC_BYTES = 41.912576e6 + 4.352e3 + 6.407e6
+PAGED_TRAFFIC_BYTES = 41.911808e6 + 3.84e3 + 6.407e6
 PAGED_FILES = ("attn_paged.cu", "combine.cu")
-PAGED_TRAFFIC_SOURCES = "29eef8cdbb458396"
+PAGED_TRAFFIC_SOURCES = "c583c6f50bf8175e"
 # the same kind of capture for the jagged prefill attention kernel
 PREFILL_TRAFFIC_BYTES = 63.266816e6 + 13.527552e6
 PREFILL_TRAFFIC_SOURCES = "2e9b4de20c6400aa"     # hash of attn_tc.cu
 # long-history attention kernel: DRAM bytes of one call on the batch's first 8 users (the capture
-# size rule), 383.73 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
+# size rule), 385.03 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
 # by that ratio (traffic grows with the pages read)
-LONG_TRAFFIC_RATIO = 383.73e6 / 371602680
+LONG_TRAFFIC_RATIO = 385.03e6 / 371602680
 # backward dQ/drab kernel (the call's dominant kernel) on the prefill batch, per launch
-BWD_DQ_TRAFFIC_BYTES = 85.321728e6 + 14.979584e6
-BWD_TRAFFIC_SOURCES = "6f745963191d2a2d"       # hash of attn_bwd_tc.cu
+BWD_DQ_TRAFFIC_BYTES = 85.2928e6 + 14.046464e6
+BWD_TRAFFIC_SOURCES = "c7a08fcd774145f8"       # hash of attn_bwd_tc.cu
 # projection GEMM (640 x 2048 x 512, SiLU) per launch
 GEMM_TRAFFIC_BYTES = 2.768384e6
-GEMM_TRAFFIC_SOURCES = "86b819eb358a215d"      # hash of gemm.cu
+GEMM_TRAFFIC_SOURCES = "08bb663a09804cd0"      # hash of gemm.cu
 
 
 def kernel_sources_hash(files) -> str:
@@ -407,7 +407,7 @@ def bench_long_history(hb, device, steps, warmup, peaks, with_cpu):
                          "traffic": (LONG_TRAFFIC_RATIO * nbytes
                                      if kernel_sources_hash(PAGED_FILES) == PAGED_TRAFFIC_SOURCES else None),
                          "traffic_note": "ncu DRAM bytes of the attention kernel on the first 8 users, scaled to "
-                                         "the full call by algorithmic bytes (1.03x algorithmic)"},
+                                         "the full call by algorithmic bytes (1.04x algorithmic)"},
             "l2": "inputs larger than L2 (1.69 GB of distinct pages per call)"}
     if with_cpu:
         import oracle
@@ -567,7 +567,7 @@ def bench_backward(hb, device, steps, warmup, peaks, with_cpu):
                                  "the call also recomputes o with the forward kernels and runs the LayerNorm backward",
                          "traffic": (BWD_DQ_TRAFFIC_BYTES if kernel_sources_hash(("attn_bwd_tc.cu",)) ==
                                      BWD_TRAFFIC_SOURCES else None),
-                         "traffic_kernel": "bwd_dq_kernel (51 % of the call in the ncu launch list) per launch"},
+                         "traffic_kernel": "bwd_dq_kernel (48 % of the call in the ncu launch list) per launch"},
             "launches_per_call": 5}
     if with_cpu:
         from oracle.dense_bwd import jagged_bwd_dense
