@@ -3,7 +3,7 @@
 //
 // What it computes (per user b, head h): for a block of 128 query rows and the key tiles the
 // block may see,
-//     S = Q K^T                               tcgen05.mma (A, B in shared memory), S in TMEM
+//     S = Q K^T                               tcgen05.mma (A = Q in TMEM, B = K in smem), S in TMEM
 //     P = allowed ? SiLU(S + rab[h][bucket(i-j)]) : 0      registers -> bf16 P in TMEM
 //     O += P V                                tcgen05.mma (A = P in TMEM, B = V in smem)
 //     O / n_max -> workspace (fp32)
@@ -16,28 +16,33 @@
 //               Q K^T has read it).
 //   warp 3      TMA producer of the V tiles (3-stage ring, freed after P V).
 //   warp 1      allocates all 512 TMEM columns; lane 0 issues every MMA:
-//               S_t = Q K_t^T into S buffer t%2, then O += P_{t-1} V_{t-1}, so the pointwise
-//               work on S_t overlaps the P V product of the previous tile.
-//   warp 2      idle after the set-up
-//   warps 4-11  for every tile they first write the 255 distinct values rab[h][bucket(i-j)]/2
-//               the tile needs (one per thread) into a double-buffered window, in four copies
-//               shifted by one float so each thread reads 16-byte vectors; a single producer
-//               warp sharing an SM sub-partition with pointwise warps paced the whole pipeline.
-//               Two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
+//               S_t = Q K_t^T, then O += P_{t-1} V_{t-1}.  One S buffer: the pointwise warps
+//               move S_t into registers first, so S_{t+1} is computed while they work on S_t.
+//               Both products take A from TMEM (Q, P) and only B from shared memory, which
+//               leaves shared-memory bandwidth to the pointwise warps while a product runs (a
+//               product with both operands in shared memory takes all of it).
+//   warp 2      bias windows: for every tile the 255 distinct values rab[h][bucket(i-j)]/2 the
+//               tile needs (eight per lane, their binary searches interleaved), in four copies
+//               shifted by one float so each reader gets 16-byte vectors, into a ring of four
+//               windows (mbarriers full / empty), up to four tiles ahead of the pointwise warps;
+//               with the second bias also the tile's key timestamps.
+//   warps 4-11  Two warpgroups; warpgroup g owns key columns [64g, 64g+64) of every tile,
 //               warp w%4 owns TMEM lanes (= query rows) [32(w%4), +32).  They load S from
 //               TMEM, form x/2 = S/2 + rab/2 with packed fp32x2 FMAs, mask, compute
 //               SiLU(x) = x/2 * (1 + tanh(x/2)), and store it as bf16 P into TMEM (P buffer
 //               t%2), where the P V MMA reads it.  The 1/n_max scale is applied to O once,
-//               when it leaves TMEM.
+//               when it leaves TMEM.  At the start warpgroup 0 copies the Q tile from shared
+//               memory into TMEM (row r -> lane r, two bf16 per column).
 //   epilogue    O / n_max leaves TMEM row per thread into a padded fp32 tile in the (then
 //               idle) K and V rings; each pointwise warp then stores whole 512-byte rows.
 // Grid: (head, user) x query block, heaviest query blocks first.  With
 // HSTU_FLAG_OVERLAP_PREVIOUS the grid is a programmatic dependent of the previous kernel: the
 // set-up runs early, and every access to inputs or the workspace -- the status word included --
 // waits for that kernel (griddepcontrol.wait).
-// TMEM columns: S0 [0,128) | S1 [128,256) | O [256,384) | P0 [384,448) | P1 [448,512)
+// TMEM columns: S [0,128) | O [128,256) | P0 [256,320) | P1 [320,384) | Q [384,448)
 // Shared memory (1024-byte aligned, 128B swizzle for every MMA operand):
-//   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 2 bias windows | bucket bounds | rab | mbarriers
+//   Q 32 KB | K 2 x 32 KB | V 3 x 32 KB | 4 bias windows | bucket bounds | rab | key timestamps
+//   | mbarriers
 // Every wait is bounded (HSTU_DEV_TIMEOUT) so a logic error cannot hang the GPU.
 #include <atomic>
 
@@ -62,19 +67,20 @@ constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
 constexpr uint32_t kWinPad = 4;               // floats before each shifted copy (stores at y - s >= -3)
 constexpr uint32_t kWinStride = 264;          // floats per copy: pad + 256 + 4 (spreads banks)
 constexpr uint32_t kWinBuf = 4 * kWinStride * 4;
+constexpr int kWinRing = 4;                   // bias windows (and key timestamps) in flight
 constexpr uint32_t kOffWin = kOffV + kVStages * kTileBytes;
-constexpr uint32_t kOffBounds = kOffWin + 2 * kWinBuf;
+constexpr uint32_t kOffBounds = kOffWin + kWinRing * kWinBuf;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr int kMaxNBT = 64;                   // time buckets (second bias)
 constexpr uint32_t kOffRabT = kOffRab + kMaxNB * 4;
-constexpr uint32_t kOffTs = kOffRabT + kMaxNBT * 4;           // key timestamps of a tile, two buffers
-constexpr uint32_t kOffBar = kOffTs + 2 * kTile * 4;
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 2 + 1;
+constexpr uint32_t kOffTs = kOffRabT + kMaxNBT * 4;           // key timestamps of a tile, one per window
+constexpr uint32_t kOffBar = kOffTs + kWinRing * kTile * 4;
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 1 + 1 + 2 + 2 + 1 + 1 + 2 * kWinRing;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemUsed = kOffMisc + 16;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;     // slack to align the base to 1024
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr uint32_t kColS = 0, kColO = 128, kColP0 = 256, kColP1 = 320, kColQ = 384;
 
 constexpr uint32_t kOStride = kTcD + 4;       // floats per row of the staged O tile (epilogue)
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -244,11 +250,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint64_t* k_empty = k_full + kKStages;      // [kKStages]
     uint64_t* v_full = k_empty + kKStages;      // [kVStages]
     uint64_t* v_empty = v_full + kVStages;      // [kVStages]
-    uint64_t* s_full = v_empty + kVStages;      // [2]
-    uint64_t* s_empty = s_full + 2;             // [2]
-    uint64_t* p_full = s_empty + 2;             // [2]
+    uint64_t* s_full = v_empty + kVStages;
+    uint64_t* s_empty = s_full + 1;
+    uint64_t* p_full = s_empty + 1;             // [2]
     uint64_t* p_empty = p_full + 2;             // [2]
     uint64_t* o_full = p_empty + 2;
+    uint64_t* qt_full = o_full + 1;             // Q copied into TMEM
+    uint64_t* win_full = qt_full + 1;           // [kWinRing] bias window t % kWinRing built
+    uint64_t* win_empty = win_full + kWinRing;  // [kWinRing] ... and read by every pointwise thread
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
     float* win = reinterpret_cast<float*>(smem + kOffWin);
@@ -267,13 +276,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
+        mbar_init(s_full, 1);
+        mbar_init(s_empty, 256);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], 256);
             mbar_init(&p_full[s], 256);
             mbar_init(&p_empty[s], 1);
         }
         mbar_init(o_full, 1);
+        mbar_init(qt_full, 128);
+        for (int s = 0; s < kWinRing; ++s) {
+            mbar_init(&win_full[s], 32);
+            mbar_init(&win_empty[s], 256);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -334,8 +348,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ============================================================ MMA issuer
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-        const uint32_t qbase = sbase + kOffQ;
-        bool ok = mbar_wait(q_full, 0, abort_flag, tmo);
+        bool ok = mbar_wait(qt_full, 0, abort_flag, tmo);
         auto issue_pv = [&](int u) -> bool {
             const int vst = u % kVStages;
             const int pb = u & 1;
@@ -357,12 +370,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         };
         for (int t = 0; ok && t < n; ++t) {
             const int kst = t % kKStages;
-            const int sb = t & 1;
             if (!mbar_wait(&k_full[kst], (t / kKStages) & 1, abort_flag, tmo)) {
                 ok = false;
                 break;
             }
-            if (t >= 2 && !mbar_wait(&s_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo)) {
+            // the S buffer is free once the pointwise warps hold S(t-1) in registers
+            if (t >= 1 && !mbar_wait(s_empty, (t - 1) & 1, abort_flag, tmo)) {
                 ok = false;
                 break;
             }
@@ -370,11 +383,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t kbase = sbase + kOffK + kst * kTileBytes;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t ad = smem_desc_sw128(qbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
+                // 16 head-dim channels per step: A = Q from TMEM (8 columns of bf16 pairs),
+                // B = K tile (keys x D, 128-byte rows) from shared memory
                 const uint64_t bd = smem_desc_sw128(kbase + (kk >> 2) * kHalf + (kk & 3) * 32, 16, 1024);
-                umma_bf16_ss(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                umma_bf16_ts(tmem + kColS, tmem + kColQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&s_full[sb]);
+            umma_commit(s_full);
             umma_commit(&k_empty[kst]);
             if (t >= 1 && !issue_pv(t - 1)) {
                 ok = false;
@@ -388,23 +402,63 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         umma_commit(o_full);
         volatile int never = 0;
         mbar_wait(o_full, 0, &never, drain);
-    } else if (warp >= 4) {
-        // ============================================================ pointwise + epilogue
-        const int pt = threadIdx.x - 128;                 // 0..255
+    } else if (warp == 2) {
+        // ============================================================ bias windows
         // rab[h]/2 and the bucket bounds (from the host, or evaluated here for many buckets)
-        for (int k = pt; k < a.NB; k += 256)
+        for (int k = lane; k < a.NB; k += 32)
             s_rab[k] = 0.5f * a.rab[(int64_t)h * a.NB + k];
-        if (kTime)
-            for (int k = pt; k < a.NBT; k += 256)
-                s_rabt[k] = 0.5f * a.rab_time[(int64_t)h * a.NBT + k];
-        for (int k = pt; k <= a.NB; k += 256)
+        for (int k = lane; k <= a.NB; k += 32)
             s_bounds[k] = bb.count > 0 ? bb.v[k]
                                        : (k == 0 ? 0 : (k == a.NB ? 0x7fffffff : bucket_bound(k, a.ln_nmax, a.NB)));
-        named_barrier_sync(2, 256);
+        __syncwarp();
         const int nb = a.NB;
         int top = 1;
         while (top * 2 <= nb)
             top *= 2;
+        // window t holds the 255 values rab[h][bucket(d)]/2 the tile needs: window index y <->
+        // distance d = (i0 - j0 + 127) - y, so query row r and key column c meet at y =
+        // 127 - r + c.  Copy s holds the window shifted by s floats after a 4-float pad, so
+        // every reader gets 16-byte aligned vectors.  Eight values per lane, searched together
+        // so their load latencies overlap; the ring lets this warp run up to four tiles ahead.
+        for (int t = 0; t < n; ++t) {
+            const int wb = t % kWinRing;
+            if (t >= kWinRing && !mbar_wait_warp(&win_empty[wb], ((t / kWinRing) & 1) ^ 1, abort_flag, tmo))
+                break;
+            const TileGeo tg = tile_geo(t, g.L);
+            float* wbuf = win + wb * (kWinBuf / 4);
+            const int32_t dist0 = i0 - tg.j0 + (kTile - 1);
+            int32_t d[8];
+            int k[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                d[e] = dist0 - (lane + 32 * e);
+            bucket_search<8>(s_bounds, nb, top, d, k);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int y = lane + 32 * e;
+                const float val = ((y <= 2 * kTile - 2) & (d[e] >= 0)) ? s_rab[k[e]] : 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    wbuf[c * kWinStride + kWinPad + (y - c)] = val;
+            }
+            if (kTime) {
+                // the tile's key timestamps (0 past the user's keys)
+#pragma unroll
+                for (int e = 0; e < kTile / 32; ++e) {
+                    const int32_t j = tg.j0 + lane + 32 * e;
+                    s_ts[wb * kTile + lane + 32 * e] = j < g.L ? a.ts[g.key_row0 + j] : 0;
+                }
+            }
+            mbar_arrive(&win_full[wb]);
+        }
+    } else if (warp >= 4) {
+        // ============================================================ pointwise + epilogue
+        const int pt = threadIdx.x - 128;                 // 0..255
+        if (kTime) {
+            for (int k = pt; k < a.NBT; k += 256)
+                s_rabt[k] = 0.5f * a.rab_time[(int64_t)h * a.NBT + k];
+            named_barrier_sync(2, 256);
+        }
         const int wg = (warp - 4) >> 2;                   // key-column half
         const int r = ((warp & 3) << 5) + lane;           // query row in the block (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -418,62 +472,67 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int wsel = y0 & 3;
         const int woff = wsel * kWinStride + kWinPad + (y0 - wsel);
         bool ok = true;
-        for (int t = 0; t < n; ++t) {
+        if (wg == 0) {
+            // Q into TMEM for the Q K^T products: row r of the tile (128-byte swizzle: the
+            // 16-byte chunk c of a row sits at chunk c ^ (r & 7)) goes to lane r, head-dim
+            // channels (2c, 2c+1) to column c, the lower channel in the low half
+            ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, tmo));
+            if (ok) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint8_t* qrow = smem + kOffQ + hf * kHalf + r * 128;
+                    uint32_t qv[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 x = *reinterpret_cast<const uint4*>(qrow + ((c ^ (r & 7)) << 4));
+                        qv[4 * c] = x.x;
+                        qv[4 * c + 1] = x.y;
+                        qv[4 * c + 2] = x.z;
+                        qv[4 * c + 3] = x.w;
+                    }
+                    tmem_st_32x32b_x32(tmem + lane_base + kColQ + hf * 32, qv);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(qt_full);
+            }
+        }
+        for (int t = 0; ok && t < n; ++t) {
             const int vst = t % kVStages;
             const int sb = t & 1;
+            const int wb = t % kWinRing;
             const TileGeo tg = tile_geo(t, g.L);
-            // the tile's bias window, one of its 255 values per pointwise thread: window index y <->
-            // distance d = (i0 - j0 + 127) - y, so query row r and key column c meet at y =
-            // 127 - r + c; copy s holds the window shifted by s floats after a 4-float pad, so every
-            // reader gets 16-byte aligned vectors.  Two buffers: the barrier below also orders this
-            // write after every read of the buffer two tiles ago.
-            float* wbuf = win + sb * (kWinBuf / 4);
-            if (kTime && pt < kTile) {
-                // the tile's key timestamps (buffer sb; ordered like the window by the barrier below)
-                const int32_t j = tg.j0 + pt;
-                s_ts[sb * kTile + pt] = j < g.L ? a.ts[g.key_row0 + j] : 0;
-            }
-            {
-                int32_t d[1] = {i0 - tg.j0 + (kTile - 1) - pt};
-                int k[1];
-                bucket_search<1>(s_bounds, nb, top, d, k);
-                const float val = ((pt <= 2 * kTile - 2) & (d[0] >= 0)) ? s_rab[k[0]] : 0.f;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    wbuf[c * kWinStride + kWinPad + (pt - c)] = val;
-            }
-            // all eight pointwise warps take this barrier once per tile, also after a timed-out
-            // wait (the rest of the iteration is then skipped, never left early)
-            named_barrier_sync(4, 256);
-            ok = ok && mbar_wait_warp(&s_full[sb], (t >> 1) & 1, abort_flag, tmo);
+            ok = mbar_wait_warp(&win_full[wb], (t / kWinRing) & 1, abort_flag, tmo) &&
+                 mbar_wait_warp(s_full, t & 1, abort_flag, tmo);
             if (!ok)
-                continue;
+                break;
             tc_fence_after();
-            const float4* wv = reinterpret_cast<const float4*>(wbuf + woff);
+            const float4* wv = reinterpret_cast<const float4*>(win + wb * (kWinBuf / 4) + woff);
             const bool full = (qrow0 + kTile - 1 < g.N) && (tg.j0 + kTile - 1 < tg.kvend) &&
                               (tg.j0 + kTile - 1 <= i0) && (tg.j0 + kTile - 1 < g.hist);
             const int32_t lim = min(lim_row, tg.kvend);
             const int32_t diag = row_valid ? i_abs : -1;
             const int jc0 = tg.j0 + wg * 64;                  // key position of column 0 of this half
-            const uint32_t scol = tmem + lane_base + (sb ? kColS1 : kColS0) + wg * 64;
+            const uint32_t scol = tmem + lane_base + kColS + wg * 64;
             uint32_t sv[32], sv2[32];
             uint32_t packed[32];
-            // first 32 columns: load, wait; then start the second load and compute the first half
+            // both halves of this thread's 64 columns into registers, then the S buffer is
+            // released: S(t+1) is computed while this tile's SiLU runs
             tmem_ld_32x32b_x32(scol, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_wait_ld();
             tmem_ld_32x32b_x32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv2[0]));
-            const int32_t* tsk = s_ts + sb * kTile + wg * 64;
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(s_empty);
+            const int32_t* tsk = s_ts + wb * kTile + wg * 64;
             if (full)
                 silu_cols32<false, kTime>(sv, wv, packed, jc0, lim, diag, ts_row, tsk, s_rabt, a.NBT);
             else
                 silu_cols32<true, kTime>(sv, wv, packed, jc0, lim, diag, ts_row, tsk, s_rabt, a.NBT);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&s_empty[sb]);
             if (full)
                 silu_cols32<false, kTime>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag, ts_row, tsk + 32, s_rabt, a.NBT);
             else
                 silu_cols32<true, kTime>(sv2, wv + 8, packed + 16, jc0 + 32, lim, diag, ts_row, tsk + 32, s_rabt, a.NBT);
+            mbar_arrive(&win_empty[wb]);                       // done with this window
             // P buffer sb is free once P V of tile t - 2 completed
             if (t >= 2) {
                 ok = ok && mbar_wait_warp(&p_empty[sb], ((t >> 1) & 1) ^ 1, abort_flag, tmo);

@@ -94,13 +94,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Whole-warp wait: lane 0 polls, the others sleep in __syncwarp; the warp leaves converged
-// and, through __syncwarp's memory ordering, with lane 0's acquire visible to every lane.
-// Polling from one lane instead of 32 keeps the shared-memory pipe free for the warps that
-// are working.
+// Non-blocking test of a phase (acquire semantics when it reports completion).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Whole-warp wait.  Fast path: every lane tests the phase (one broadcast access for the warp)
+// and a vote decides, so a phase that has already completed costs no divergence.  Otherwise
+// lane 0 waits (sleeping between polls), the others wait in __syncwarp; the warp leaves
+// converged and, through __syncwarp's memory ordering, with lane 0's acquire visible to every
+// lane.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                uint64_t limit_ns)
 {
+    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity)))
+        return true;
     bool ok = true;
     if ((threadIdx.x & 31) == 0)
         ok = mbar_wait(bar, parity, abort, limit_ns);
