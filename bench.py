@@ -39,32 +39,37 @@ METRIC = "HSTU paged-attn new tokens/s per B200; % of BF16 tensor / HBM roofline
 # batch, from one `ncu --set full` capture of the attention and LayerNorm kernels (ncu flushes
 # caches, so the LayerNorm kernel's partial-plane reads show up as DRAM reads).  Valid only for
 # the kernel sources they were taken from (hash below); otherwise the bench reports traffic as null.
-PAGED_TRAFFIC_BYTES = 41.911808e6 + 3.84e3 + 6.407e6
+PAGED_TRAFFIC_BYTES = 41.913088e6 + 4.096e3 + 6.407e6
 PAGED_FILES = ("attn_paged.cu", "combine.cu")
-PAGED_TRAFFIC_SOURCES = "c583c6f50bf8175e"
+PAGED_TRAFFIC_SOURCES = "6ba38f878f0500ea"
 # the same kind of capture for the jagged prefill attention kernel
-PREFILL_TRAFFIC_BYTES = 63.266816e6 + 13.527552e6
-PREFILL_TRAFFIC_SOURCES = "2e9b4de20c6400aa"     # hash of attn_tc.cu
+PREFILL_TRAFFIC_BYTES = 63.340032e6 + 12.201472e6
+PREFILL_TRAFFIC_SOURCES = "4b6330fe5376419d"
 # long-history attention kernel: DRAM bytes of one call on the batch's first 8 users (the capture
-# size rule), 385.03 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
+# size rule), 381.17 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
 # by that ratio (traffic grows with the pages read)
-LONG_TRAFFIC_RATIO = 385.03e6 / 371602680
+LONG_TRAFFIC_RATIO = 381.17e6 / 371602680
 # backward dQ/drab kernel (the call's dominant kernel) on the prefill batch, per launch
-BWD_DQ_TRAFFIC_BYTES = 85.2928e6 + 14.046464e6
-BWD_TRAFFIC_SOURCES = "c7a08fcd774145f8"       # hash of attn_bwd_tc.cu
+BWD_DQ_TRAFFIC_BYTES = 85.454848e6 + 13.673472e6
+BWD_TRAFFIC_SOURCES = "4e6d1ec2dcdb68ae"       # hash of attn_bwd_tc.cu
 # projection GEMM (640 x 2048 x 512, SiLU) per launch
-GEMM_TRAFFIC_BYTES = 2.768384e6
-GEMM_TRAFFIC_SOURCES = "08bb663a09804cd0"      # hash of gemm.cu
+GEMM_TRAFFIC_BYTES = 2.769e6
+GEMM_TRAFFIC_SOURCES = "65ee9d0fc18e6424"      # hash of gemm.cu
+
+
+# headers every kernel includes (wait loops, descriptors, argument blocks)
+SHARED_KERNEL_HEADERS = ("sm100.cuh", "common.cuh", "kernels.cuh")
 
 
 def kernel_sources_hash(files) -> str:
-    """Hash of the kernels' source code with comments and blank space removed (editing a comment
-    does not change the kernel the counters were taken from)."""
+    """Hash of the kernels' source code (the listed files and the shared headers) with comments
+    and blank space removed (editing a comment does not change the kernel the counters were
+    taken from)."""
     import hashlib
     import re
 
     h = hashlib.sha256()
-    for f in files:
+    for f in tuple(files) + SHARED_KERNEL_HEADERS:
         with open(os.path.join(ROOT, "hstu_attention_b200", "csrc", f), encoding="utf-8") as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -407,7 +412,7 @@ def bench_long_history(hb, device, steps, warmup, peaks, with_cpu):
                          "traffic": (LONG_TRAFFIC_RATIO * nbytes
                                      if kernel_sources_hash(PAGED_FILES) == PAGED_TRAFFIC_SOURCES else None),
                          "traffic_note": "ncu DRAM bytes of the attention kernel on the first 8 users, scaled to "
-                                         "the full call by algorithmic bytes (1.04x algorithmic)"},
+                                         "the full call by algorithmic bytes (1.03x algorithmic)"},
             "l2": "inputs larger than L2 (1.69 GB of distinct pages per call)"}
     if with_cpu:
         import oracle
