@@ -13,23 +13,26 @@
 // statistics, so both kernels below recompute S tile by tile and need nothing else.
 //
 // bwd_dq_kernel   one CTA per (user, head, 128-query block), grid and order as the forward:
-//                 per key tile  S = Q K^T and dP = dO V^T (tcgen05, SS), pointwise dS -> bf16 in
-//                 TMEM, dQ += dS K (tcgen05, A = dS from TMEM, B = the K tile read MN-major);
-//                 drab: dS summed along the tile's 255 diagonals (a shuffle reduction per 32 x 32
-//                 block into per-warp arrays), folded into per-CTA bucket sums, one global atomic
-//                 per bucket at the end.
+//                 per key tile  S = Q K^T (tcgen05, A = Q copied into TMEM once) and dP = dO V^T
+//                 (tcgen05, SS), pointwise dS -> bf16 in TMEM, dQ += dS K (tcgen05, A = dS from
+//                 TMEM, B = the K tile read MN-major); the next tile's S and dP are issued as soon
+//                 as the pointwise warps hold this tile's in registers.  drab: dS summed along the
+//                 tile's 255 diagonals (a shuffle reduction per 32 x 32 block into per-warp arrays,
+//                 two buffers), folded by warp 3 into per-CTA bucket sums (runs of equal buckets
+//                 summed across lanes first), one global atomic per bucket at the end.
 // bwd_dkv_kernel  one CTA per (user, head, 128-key block), the blocks with most queries first:
 //                 per query tile the transposed products S^T = K Q^T and dP^T = V dO^T, pointwise
 //                 P^T and dS^T -> bf16 in TMEM (written over the S^T / dP^T columns already read),
-//                 dV += P^T dO and dK += dS^T Q (A from TMEM, B = the dO / Q tile read MN-major).
-// Both kernels run their products and the pointwise stage one after the other per tile (the MMA
-// thread waits for the pointwise results before the products that read them, and for those
-// products before it overwrites their TMEM operands): a first tensor-core path, not yet
-// pipelined across tiles.  Every wait is bounded (HSTU_DEV_TIMEOUT).
+//                 dV += P^T dO and dK += dS^T Q (A from TMEM, B = the dO / Q tile read MN-major);
+//                 products and pointwise stage alternate per tile (TMEM is full).
+// Every wait is bounded (HSTU_DEV_TIMEOUT).
 //
 // CTA roles (384 threads): warp 0 lane 0 TMA producer; warp 1 allocates all 512 TMEM columns and
-// lane 0 issues the MMAs; warps 4-11 pointwise and epilogue (warpgroup g owns tile columns
-// [64g, 64g + 64), warp w%4 owns TMEM lanes [32(w%4), +32)).
+// lane 0 issues the MMAs; warp 2 builds each tile's bias window (255 values rab[h][bucket(i-j)],
+// eight per lane with interleaved binary searches; for the dQ kernel also the bucket index per
+// diagonal) into a two-slot ring; warp 3 (dQ kernel) folds the diagonal sums; warps 4-11
+// pointwise and epilogue (warpgroup g owns tile columns [64g, 64g + 64), warp w%4 owns TMEM lanes
+// [32(w%4), +32)), with no barrier among them inside the tile loop.
 #include <atomic>
 
 #include "common.cuh"
@@ -47,8 +50,9 @@ constexpr int kThreads = 384;
 constexpr int kMaxNB = 1024;
 constexpr uint32_t kHalf = 128 * 128;           // 128 rows x 128 bytes
 constexpr uint32_t kTileBytes = 2 * kHalf;      // a 128 x 128 bf16 operand
-// shared memory: two fixed operands (Q, dO or K, V), a 2-stage ring of operand pairs, the bias
-// window (four shifted copies), its bucket indices, diagonal sums, bucket sums, bounds, rab
+// shared memory: two fixed operands (Q, dO or K, V), a 2-stage ring of operand pairs, the
+// window area (a two-slot ring of bias windows and bucket indices), diagonal sums (buffer 0;
+// buffer 1 of the dQ kernel reuses the Q tile's space), bucket sums, bounds, rab
 constexpr uint32_t kOffFix0 = 0;
 constexpr uint32_t kOffFix1 = kTileBytes;
 constexpr uint32_t kOffRing = 2 * kTileBytes;                // 2 stages x 2 operands
@@ -62,22 +66,18 @@ constexpr uint32_t kOffBsum = kOffDiag + 8 * 256 * 4;
 constexpr uint32_t kOffBounds = kOffBsum + kMaxNB * 4;
 constexpr uint32_t kOffRab = kOffBounds + (kMaxNB + 4) * 4;
 constexpr uint32_t kOffBar = kOffRab + kMaxNB * 4;
-constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1;     // fix, ring full/empty, sp_full, pd_full, pd_empty, acc, sp_empty
+// fix, ring full/empty, sp_full, pd_full, pd_empty, acc, sp_empty; the dQ kernel adds qt_full,
+// win_full/empty [2] and diag_full/empty [2]
+constexpr int kNumBars = 1 + 2 + 2 + 1 + 1 + 1 + 1 + 1 + 1 + 2 + 2 + 2 + 2;
+// dQ kernel: bias windows in a two-slot ring (one copy each, then the bucket index per position)
+constexpr uint32_t kWinSlotFloats = 264;                    // pad + 256 + 4
+constexpr uint32_t kWinSlotBytes = kWinSlotFloats * 4 + 256 * 4;
+static_assert(2 * kWinSlotBytes <= kOffDiag - kOffWin, "window ring fits the window area");
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;
 constexpr uint32_t kTmemCols = 512;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
-
-// bucket(d) by a branchless binary search over the staged bounds (bounds[0] = 0,
-// bounds[nb] = INT_MAX, d < 0 -> 0)
-__device__ __forceinline__ int bucket_idx(const int32_t* bounds, int nb, int top, int32_t d)
-{
-    int k = 0;
-    for (int step = top; step > 0; step >>= 1)
-        k += (bounds[min(k + step, nb)] <= d) ? step : 0;
-    return k;
-}
 
 __device__ int bucket_bound_bt(int k, double ln_nmax, int nb)
 {
@@ -108,10 +108,9 @@ struct Smem {
     uint8_t* base;
     uint32_t sbase;
     uint64_t *fix_full, *ring_full, *ring_empty, *sp_full, *sp_empty, *pd_full, *pd_empty, *acc_full;
+    uint64_t *qt_full, *win_full, *win_empty, *diag_full, *diag_empty;    // dQ kernel
     uint32_t* tmem_slot;
     volatile int* abort_flag;
-    float* win;
-    int32_t* wink;
     float* diag;
     float* bsum;
     int32_t* bounds;
@@ -134,10 +133,13 @@ __device__ __forceinline__ Smem carve(uint8_t* smem_raw)
     m.pd_empty = bars + 7;
     m.acc_full = bars + 8;
     m.sp_empty = bars + 9;
+    m.qt_full = bars + 10;
+    m.win_full = bars + 11;
+    m.win_empty = bars + 13;
+    m.diag_full = bars + 15;
+    m.diag_empty = bars + 17;
     m.tmem_slot = reinterpret_cast<uint32_t*>(m.base + kOffMisc);
     m.abort_flag = reinterpret_cast<volatile int*>(m.base + kOffMisc + 4);
-    m.win = reinterpret_cast<float*>(m.base + kOffWin);
-    m.wink = reinterpret_cast<int32_t*>(m.base + kOffWinK);
     m.diag = reinterpret_cast<float*>(m.base + kOffDiag);
     m.bsum = reinterpret_cast<float*>(m.base + kOffBsum);
     m.bounds = reinterpret_cast<int32_t*>(m.base + kOffBounds);
@@ -146,9 +148,21 @@ __device__ __forceinline__ Smem carve(uint8_t* smem_raw)
 }
 
 // barrier init (thread 0) and TMEM allocation (warp 1), then a CTA barrier
-__device__ __forceinline__ uint32_t setup(const Smem& m, int warp)
+// roles: 1 = the dQ kernel (window ring read by the pointwise warps and the fold warp, diagonal
+// buffers, Q in TMEM), 2 = the dK/dV kernel (window ring read by the pointwise warps)
+__device__ __forceinline__ uint32_t setup(const Smem& m, int warp, int roles)
 {
     if (threadIdx.x == 0) {
+        if (roles == 1)
+            mbar_init(m.qt_full, 128);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&m.win_full[s], 32);
+            mbar_init(&m.win_empty[s], roles == 1 ? 256 + 32 : 256);
+            if (roles == 1) {
+                mbar_init(&m.diag_full[s], 256);
+                mbar_init(&m.diag_empty[s], 32);
+            }
+        }
         mbar_init(m.fix_full, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&m.ring_full[s], 1);
@@ -199,37 +213,6 @@ __device__ __forceinline__ void stage_bias(const Smem& m, const BwdTcArgs& a, co
         m.diag[x] = 0.f;
 }
 
-// One window position per pointwise thread: distance d(y) = dist0 + sgn * y for y = pt;
-// writes rab[bucket(d)] (0 for d < 0 or y > 254) into the four shifted copies and the bucket index.
-__device__ __forceinline__ void build_window(const Smem& m, int pt, int32_t dist0, int sgn, int nb, int top)
-{
-    const int32_t d = dist0 + sgn * pt;
-    const bool live = (pt <= 2 * kTile - 2) && d >= 0;
-    const int k = live ? bucket_idx(m.bounds, nb, top, d) : 0;
-    const float val = live ? m.rab[k] : 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        m.win[c * kWinStride + kWinPad + (pt - c)] = val;
-    m.wink[pt] = live ? k : -1;
-}
-
-// fold the tile's diagonal sums (one private array per pointwise warp) into the bucket sums and
-// clear them (after a barrier)
-__device__ __forceinline__ void fold_diagonals(const Smem& m, int pt)
-{
-    if (pt < 2 * kTile - 1) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            v += m.diag[w * 256 + pt];
-            m.diag[w * 256 + pt] = 0.f;
-        }
-        const int k = m.wink[pt];
-        if (v != 0.f && k >= 0)
-            atomicAdd(&m.bsum[k], v);
-    }
-}
-
 // ============================================================================ dQ and drab
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -264,10 +247,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int n = last_q / kTile + 1;                 // key tiles 0 .. n - 1 (keys up to last_q)
 
     const Smem m = carve(smem_raw);
-    const uint32_t tmem = setup(m, warp);
+    const uint32_t tmem = setup(m, warp, 1);
     const uint64_t tmo = a.timeout_ns, drain = a.drain_ns;
-    // TMEM: S [0,128) | dP [128,256) | dQ [256,384) | dS bf16 [384,448)
-    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256, cDS = 384;
+    // TMEM: S [0,128) | dP [128,256) | dQ [256,384) | dS bf16 [384,448) | Q bf16 [448,512)
+    constexpr uint32_t cS = 0, cDP = 128, cDQ = 256, cDS = 384, cQ = 448;
+    // diagonal sums of tile t go to buffer t & 1: buffer 0 in its own area, buffer 1 in the Q
+    // tile's space once Q has been copied into TMEM
+    float* const diag_buf[2] = {m.diag, reinterpret_cast<float*>(m.base + kOffFix0)};
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -296,10 +282,10 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_wait(&m.ring_full[t & 1], (t >> 1) & 1, &never, drain);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc_ss = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_kmaj = idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t idesc_ts = idesc_bf16_f32(128, 128, 0, 1);
-        bool ok = mbar_wait(m.fix_full, 0, m.abort_flag, tmo);
-        // S(t) = Q K_t^T and dP(t) = dO V_t^T into their TMEM columns (stage t & 1 of the ring)
+        bool ok = mbar_wait(m.fix_full, 0, m.abort_flag, tmo) && mbar_wait(m.qt_full, 0, m.abort_flag, tmo);
+        // S(t) = Q K_t^T (A = Q from TMEM) and dP(t) = dO V_t^T (both operands in shared memory)
         auto issue_sdp = [&](int t) -> bool {
             const int st = t & 1;
             const uint32_t kb = m.sbase + kOffRing + st * kStageBytes;
@@ -310,14 +296,14 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kHalf + (kk & 3) * 32;
-                umma_bf16_ss(tmem + cS, smem_desc_sw128(m.sbase + kOffFix0 + ko, 16, 1024),
-                             smem_desc_sw128(kb + ko, 16, 1024), idesc_ss, kk > 0 ? 1u : 0u);
+                umma_bf16_ts(tmem + cS, tmem + cQ + kk * 8, smem_desc_sw128(kb + ko, 16, 1024), idesc_kmaj,
+                             kk > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * kHalf + (kk & 3) * 32;
                 umma_bf16_ss(tmem + cDP, smem_desc_sw128(m.sbase + kOffFix1 + ko, 16, 1024),
-                             smem_desc_sw128(vb + ko, 16, 1024), idesc_ss, kk > 0 ? 1u : 0u);
+                             smem_desc_sw128(vb + ko, 16, 1024), idesc_kmaj, kk > 0 ? 1u : 0u);
             }
             umma_commit(m.sp_full);
             return true;
@@ -352,15 +338,100 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         umma_commit(m.acc_full);
         volatile int never = 0;
         mbar_wait(m.acc_full, 0, &never, drain);
-    } else if (warp >= 4) {
-        // ------------------------------------------------------------ pointwise + epilogue
-        const int pt = threadIdx.x - 128;
-        stage_bias(m, a, bb, h, pt);
-        named_barrier_sync(2, 256);
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ bias windows
+        // window t (slot t & 1): position y = 127 - r + c of query row r and key column c has
+        // distance d = i - j = (qrow0 - j0 + 127) - y; value rab[bucket(d)] (0 for d < 0 or
+        // y > 254) and the bucket index (-1 there) for the fold.  Eight positions per lane, their
+        // binary searches interleaved.
+        named_barrier_sync(2, 320);                        // bounds and rab staged
         const int nb = a.NB;
         int top = 1;
         while (top * 2 <= nb)
             top *= 2;
+        for (int t = 0; t < n; ++t) {
+            const int sl = t & 1;
+            if (t >= 2 && !mbar_wait_warp(&m.win_empty[sl], ((t >> 1) & 1) ^ 1, m.abort_flag, tmo))
+                break;
+            float* win = reinterpret_cast<float*>(m.base + kOffWin + sl * kWinSlotBytes);
+            int32_t* wk = reinterpret_cast<int32_t*>(m.base + kOffWin + sl * kWinSlotBytes + kWinSlotFloats * 4);
+            const int32_t dist0 = qrow0 - t * kTile + (kTile - 1);
+            int k[8];
+            int32_t d[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                d[e] = dist0 - (lane + 32 * e);
+                k[e] = 0;
+            }
+            for (int step = top; step > 0; step >>= 1) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    k[e] += (m.bounds[min(k[e] + step, nb)] <= d[e]) ? step : 0;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int y = lane + 32 * e;
+                const bool live = (y <= 2 * kTile - 2) && d[e] >= 0;
+                win[kWinPad + y] = live ? m.rab[k[e]] : 0.f;
+                wk[y] = live ? k[e] : -1;
+            }
+            mbar_arrive(&m.win_full[sl]);
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ drab fold
+        // tile t's diagonal sums (buffer t & 1, one array per pointwise warp) into the bucket
+        // sums, then the buffer is cleared for tile t + 2; one global atomic per bucket at the end
+        named_barrier_sync(2, 320);                        // bucket sums zeroed
+        bool ok = true;
+        for (int t = 0; ok && t < n; ++t) {
+            const int sl = t & 1;
+            ok = mbar_wait_warp(&m.diag_full[sl], (t >> 1) & 1, m.abort_flag, tmo);
+            if (!ok)
+                break;
+            float* db = diag_buf[sl];
+            const int32_t* wk =
+                reinterpret_cast<const int32_t*>(m.base + kOffWin + sl * kWinSlotBytes + kWinSlotFloats * 4);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int y = lane + 32 * e;
+                const bool live = y <= 2 * kTile - 2;
+                float v = 0.f;
+                if (live) {
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        v += db[w * 256 + y];
+                        db[w * 256 + y] = 0.f;
+                    }
+                }
+                const int kb = live ? wk[y] : -1;
+                // buckets do not increase along y, so equal buckets are runs of lanes: a suffix
+                // sum within each run leaves the run's total in its first lane, which alone
+                // adds it to the bucket (one shared atomic per run instead of one per lane)
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float vo = __shfl_down_sync(0xffffffffu, v, o);
+                    const int ko = __shfl_down_sync(0xffffffffu, kb, o);
+                    if (lane + o < 32 && ko == kb)
+                        v += vo;
+                }
+                const int kprev = __shfl_up_sync(0xffffffffu, kb, 1);
+                if (kb >= 0 && (lane == 0 || kprev != kb) && v != 0.f)
+                    atomicAdd(&m.bsum[kb], v);
+            }
+            __syncwarp();
+            mbar_arrive(&m.diag_empty[sl]);
+            mbar_arrive(&m.win_empty[sl]);
+        }
+        __syncwarp();
+        if (ok)
+            for (int k = lane; k < a.NB; k += 32)
+                if (m.bsum[k] != 0.f)
+                    atomicAdd(&a.drab[(int64_t)h * a.NB + k], m.bsum[k]);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ pointwise + epilogue
+        const int pt = threadIdx.x - 128;
+        stage_bias(m, a, bb, h, pt);
+        named_barrier_sync(2, 320);
         const int wg = (warp - 4) >> 2;
         const int r = ((warp & 3) << 5) + lane;            // query row (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
@@ -369,16 +440,48 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int32_t lim = row_valid ? min(i + 1, g.hist) : -1;   // keys j < lim are visible, and j == i
         const int32_t diag_key = row_valid ? i : -1;
         const float inv_n = a.inv_n;
-        float* wdiag = m.diag + (warp - 4) * 256;
         bool ok = true;
+        if (wg == 0) {
+            // Q into TMEM for the Q K^T products: row r of the tile (128-byte swizzle: the 16-byte
+            // chunk c of a row sits at chunk c ^ (r & 7)) goes to lane r, channels (2c, 2c+1) to
+            // column c; then the tile's space is cleared for diagonal buffer 1
+            ok = __all_sync(0xffffffffu, mbar_wait(m.fix_full, 0, m.abort_flag, tmo));
+            if (ok) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint8_t* qrow = m.base + kOffFix0 + hf * kHalf + r * 128;
+                    uint32_t qv[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 x = *reinterpret_cast<const uint4*>(qrow + ((c ^ (r & 7)) << 4));
+                        qv[4 * c] = x.x;
+                        qv[4 * c + 1] = x.y;
+                        qv[4 * c + 2] = x.z;
+                        qv[4 * c + 3] = x.w;
+                    }
+                    tmem_st_32x32b_x32(tmem + lane_base + cQ + hf * 32, qv);
+                }
+                tmem_wait_st();
+            }
+            named_barrier_sync(5, 128);                    // every row of Q has been read
+            for (int x = pt; x < 8 * 256; x += 128)
+                diag_buf[1][x] = 0.f;
+            tc_fence_before();
+            mbar_arrive(m.qt_full);
+        }
+        // diagonal buffer 1 is cleared and Q is in TMEM
+        ok = ok && mbar_wait_warp(m.qt_full, 0, m.abort_flag, tmo);
         for (int t = 0; t < n; ++t) {
             const int32_t j0 = t * kTile;
-            // window position y = 127 - r + c <-> distance d = i - j = (qrow0 - j0 + 127) - y
-            build_window(m, pt, qrow0 - j0 + (kTile - 1), -1, nb, top);
-            named_barrier_sync(4, 256);
-            ok = ok && mbar_wait_warp(m.sp_full, t & 1, m.abort_flag, tmo);
+            const int sl = t & 1;
+            ok = ok && mbar_wait_warp(&m.win_full[sl], (t >> 1) & 1, m.abort_flag, tmo) &&
+                 mbar_wait_warp(m.sp_full, t & 1, m.abort_flag, tmo);
+            if (ok && t >= 2)
+                ok = mbar_wait_warp(&m.diag_empty[sl], ((t >> 1) & 1) ^ 1, m.abort_flag, tmo);
             if (ok) {
                 tc_fence_after();
+                const float* win = reinterpret_cast<const float*>(m.base + kOffWin + sl * kWinSlotBytes);
+                float* wdiag = diag_buf[sl] + (warp - 4) * 256;
                 const int y0 = (kTile - 1) - r + 64 * wg;
 #pragma unroll 1
                 for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -404,7 +507,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const int c = 64 * wg + c0 + e + q;
                             const int32_t j = j0 + c;
                             const int y = y0 + c0 + e + q;
-                            const float s = __uint_as_float(sv[e + q]) + m.win[kWinPad + y];
+                            const float s = __uint_as_float(sv[e + q]) + win[kWinPad + y];
                             float p;
                             const float ds = pair_terms(s, __uint_as_float(dv[e + q]), inv_n, p);
                             const bool allowed = (j < lim) | (j == diag_key);
@@ -436,14 +539,12 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             __syncwarp();
             tmem_wait_st();
-            named_barrier_sync(4, 256);                    // diagonal sums complete
-            fold_diagonals(m, pt);
             if (ok) {
                 tc_fence_before();
                 mbar_arrive(m.pd_full);
+                mbar_arrive(&m.diag_full[sl]);             // this tile's diagonal sums are complete
+                mbar_arrive(&m.win_empty[sl]);             // and its window has been read
             }
-            __syncwarp();
-            named_barrier_sync(4, 256);                    // window and diagonals reusable
         }
         // ------------------------------------------------------------ epilogue
         // tcgen05.ld is a warp-wide instruction: every lane loads, only the rows of queries store
@@ -466,11 +567,6 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 __syncwarp();
             }
         }
-        named_barrier_sync(4, 256);
-        if (ok)
-            for (int k = pt; k < nb; k += 256)
-                if (m.bsum[k] != 0.f)
-                    atomicAdd(&a.drab[(int64_t)h * nb + k], m.bsum[k]);
     }
     teardown(m, warp, tmem, a.ws);
 }
@@ -507,7 +603,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int n = nq_tiles - t0;
 
     const Smem m = carve(smem_raw);
-    const uint32_t tmem = setup(m, warp);
+    const uint32_t tmem = setup(m, warp, 2);
     const uint64_t tmo = a.timeout_ns, drain = a.drain_ns;
     // TMEM: S^T [0,128) (P^T bf16 written over it) | dP^T [128,256) (dS^T over it) | dV | dK
     constexpr uint32_t cS = 0, cDP = 128, cDV = 256, cDK = 384;
@@ -592,14 +688,45 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         umma_commit(m.acc_full);
         volatile int never = 0;
         mbar_wait(m.acc_full, 0, &never, drain);
-    } else if (warp >= 4) {
-        const int pt = threadIdx.x - 128;
-        stage_bias(m, a, bb, h, pt);
-        named_barrier_sync(2, 256);
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ bias windows
+        // window t (slot t & 1): position y = 127 - r + c of key row r and query column c has
+        // distance d = i - j = (i0 - j0 - 127) + y; value rab[bucket(d)] (0 for d < 0 or
+        // y > 254).  Eight positions per lane, their binary searches interleaved.
+        named_barrier_sync(2, 288);                        // bounds and rab staged
         const int nb = a.NB;
         int top = 1;
         while (top * 2 <= nb)
             top *= 2;
+        for (int t = 0; t < n; ++t) {
+            const int sl = t & 1;
+            if (t >= 2 && !mbar_wait_warp(&m.win_empty[sl], ((t >> 1) & 1) ^ 1, m.abort_flag, tmo))
+                break;
+            float* win = reinterpret_cast<float*>(m.base + kOffWin + sl * kWinSlotBytes);
+            const int32_t dist0 = (t0 + t) * kTile - j0 - (kTile - 1);
+            int k[8];
+            int32_t d[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                d[e] = dist0 + (lane + 32 * e);
+                k[e] = 0;
+            }
+            for (int step = top; step > 0; step >>= 1) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    k[e] += (m.bounds[min(k[e] + step, nb)] <= d[e]) ? step : 0;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int y = lane + 32 * e;
+                win[kWinPad + y] = ((y <= 2 * kTile - 2) && d[e] >= 0) ? m.rab[k[e]] : 0.f;
+            }
+            mbar_arrive(&m.win_full[sl]);
+        }
+    } else if (warp >= 4) {
+        const int pt = threadIdx.x - 128;
+        stage_bias(m, a, bb, h, pt);
+        named_barrier_sync(2, 288);
         const int wg = (warp - 4) >> 2;
         const int r = ((warp & 3) << 5) + lane;            // key row (= TMEM lane)
         const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
@@ -612,12 +739,12 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         bool ok = true;
         for (int t = 0; t < n; ++t) {
             const int32_t i0 = (t0 + t) * kTile;
-            // window position y = 127 - r + c <-> distance d = i - j = (i0 - j0 - 127) + y
-            build_window(m, pt, i0 - j0 - (kTile - 1), 1, nb, top);
-            named_barrier_sync(4, 256);
-            ok = ok && mbar_wait_warp(m.sp_full, t & 1, m.abort_flag, tmo);
+            const int sl = t & 1;
+            ok = ok && mbar_wait_warp(&m.win_full[sl], (t >> 1) & 1, m.abort_flag, tmo) &&
+                 mbar_wait_warp(m.sp_full, t & 1, m.abort_flag, tmo);
             if (ok) {
                 tc_fence_after();
+                const float* win = reinterpret_cast<const float*>(m.base + kOffWin + sl * kWinSlotBytes);
                 const int y0 = (kTile - 1) - r + 64 * wg;
 #pragma unroll 1
                 for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -634,7 +761,7 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             const int c = 64 * wg + c0 + e + q;
                             const int32_t i = i0 + c;
                             const int y = y0 + c0 + e + q;
-                            const float s = __uint_as_float(sv[e + q]) + m.win[kWinPad + y];
+                            const float s = __uint_as_float(sv[e + q]) + win[kWinPad + y];
                             float p;
                             const float ds = pair_terms(s, __uint_as_float(dv[e + q]), inv_n, p);
                             const bool allowed = (i < g.N) & ((i >= lo) | (i == self));
@@ -657,8 +784,8 @@ bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (ok) {
                 tc_fence_before();
                 mbar_arrive(m.pd_full);
+                mbar_arrive(&m.win_empty[sl]);             // this tile's window has been read
             }
-            named_barrier_sync(4, 256);                    // the window is reusable
         }
         // warp-wide TMEM loads, per-lane stores (only the rows of keys of the user)
         ok = ok && mbar_wait_warp(m.acc_full, 0, m.abort_flag, tmo);
