@@ -50,8 +50,8 @@ PREFILL_TRAFFIC_SOURCES = "4b6330fe5376419d"
 # by that ratio (traffic grows with the pages read)
 LONG_TRAFFIC_RATIO = 381.17e6 / 371602680
 # backward dQ/drab kernel (the call's dominant kernel) on the prefill batch, per launch
-BWD_DQ_TRAFFIC_BYTES = 85.454848e6 + 13.673472e6
-BWD_TRAFFIC_SOURCES = "4e6d1ec2dcdb68ae"       # hash of attn_bwd_tc.cu
+BWD_DQ_TRAFFIC_BYTES = 85.852928e6 + 13.68832e6
+BWD_TRAFFIC_SOURCES = "59548f9c264f2571"       # hash of attn_bwd_tc.cu
 # projection GEMM (640 x 2048 x 512, SiLU) per launch
 GEMM_TRAFFIC_BYTES = 2.769e6
 GEMM_TRAFFIC_SOURCES = "65ee9d0fc18e6424"      # hash of gemm.cu
